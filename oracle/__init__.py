@@ -1,0 +1,10 @@
+"""CPU float64 oracle for the exact attention forward.
+
+TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
+and the CPU-baseline leg of ``bench.py``.  The CUDA path never imports it.
+"""
+from .attention import (  # noqa: F401
+    apply_causal_mask, attention_f64, attention_head_rows, attention_probs_f64,
+    brute_force, logsumexp_rows, online_softmax_f64, scores, softmax_rows,
+    to_f64, weighted_sum,
+)
