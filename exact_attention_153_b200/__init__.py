@@ -1,0 +1,195 @@
+"""Python binding of the sm_100a exact attention forward (libattn_sm100.so).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+library.  PyTorch supplies device memory and streams.  If the library is not
+built the import still works, but every call raises -- there is no CPU or
+PyTorch fallback.
+
+    from exact_attention_153_b200 import forward
+    o, lse = forward(q, k, v, causal=True)          # q, k, v: [B, H, N, d] cuda fp16/bf16
+
+The C entry points are mirrored one to one (``attn_fwd``, ``attn_fwd_host``,
+``attn_plan``, ``attn_get_device_status``, ``attn_strerror``,
+``attn_version``) for callers that manage raw pointers.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = [
+    "ATTN_FP16", "ATTN_BF16", "AttnError", "lib", "library_path", "attn_fwd", "attn_fwd_host",
+    "attn_plan", "attn_get_device_status", "attn_strerror", "attn_version", "forward",
+    "forward_host", "STATUS_NAMES",
+]
+
+ATTN_FP16 = 0
+ATTN_BF16 = 1
+STATUS_NAMES = {
+    0: "ATTN_OK", 1: "ATTN_ERR_NULL", 2: "ATTN_ERR_SHAPE", 3: "ATTN_ERR_HEAD_DIM",
+    4: "ATTN_ERR_DTYPE", 5: "ATTN_ERR_ALIGN", 6: "ATTN_ERR_SCALE", 7: "ATTN_ERR_ARCH",
+    8: "ATTN_ERR_CUDA", 9: "ATTN_ERR_DEVICE_TIMEOUT",
+}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libattn_sm100.so"
+_lib = None
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+class AttnError(RuntimeError):
+    """A non-zero status from the C library."""
+
+    def __init__(self, status: int, where: str = "attn_fwd"):
+        self.status = int(status)
+        name = STATUS_NAMES.get(self.status, str(status))
+        super().__init__(f"{where} failed: {name}: {attn_strerror(self.status)}")
+
+
+class _Plan(ctypes.Structure):
+    _fields_ = [("num_q_tiles", ctypes.c_int), ("num_q_pairs", ctypes.c_int),
+                ("num_kv_tiles", ctypes.c_int), ("num_units", ctypes.c_int),
+                ("grid", ctypes.c_int), ("block", ctypes.c_int), ("smem_bytes", ctypes.c_int),
+                ("stages", ctypes.c_int), ("qk_tile_products", ctypes.c_longlong)]
+
+
+def lib() -> ctypes.CDLL:
+    """Load the in-tree library (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        path = library_path()
+        if not os.path.exists(path):
+            raise RuntimeError(
+                f"{path} is missing: build it with `python -m exact_attention_153_b200.build_lib` "
+                "(there is no fallback implementation)")
+        L = ctypes.CDLL(path)
+        vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+        L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+        L.attn_fwd.restype = i
+        L.attn_fwd_host.argtypes = [vp] * 10 + [i, i, i, i, i, f, i, i, vp]
+        L.attn_fwd_host.restype = i
+        L.attn_plan.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(_Plan)]
+        L.attn_plan.restype = i
+        L.attn_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+        L.attn_get_device_status.restype = i
+        L.attn_strerror.argtypes = [i]
+        L.attn_strerror.restype = ctypes.c_char_p
+        L.attn_version.argtypes = []
+        L.attn_version.restype = i
+        _lib = L
+    return _lib
+
+
+# ----------------------------------------------------------------- raw entry points
+
+def attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, stream) -> int:
+    """Raw ``attn_fwd``: pointers and the stream handle as Python ints."""
+    return lib().attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, float(scale), int(causal), dtype, stream)
+
+
+def attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, B, H, Nq, Nk, d, scale,
+                  causal, dtype, stream) -> int:
+    """Raw ``attn_fwd_host``: host and device pointers as Python ints."""
+    return lib().attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, B, H, Nq,
+                               Nk, d, float(scale), int(causal), dtype, stream)
+
+
+def attn_plan(B, H, Nq, Nk, d, causal, num_sms) -> dict:
+    """Launch geometry for these sizes on a GPU with ``num_sms`` SMs."""
+    p = _Plan()
+    st = lib().attn_plan(B, H, Nq, Nk, d, int(causal), num_sms, ctypes.byref(p))
+    if st != 0:
+        raise AttnError(st, "attn_plan")
+    return {name: getattr(p, name) for name, _ in _Plan._fields_}
+
+
+def attn_get_device_status(stream=None):
+    """(status, raw word) after synchronising ``stream``."""
+    word = ctypes.c_uint(0)
+    st = lib().attn_get_device_status(_stream_handle(stream), ctypes.byref(word))
+    return st, word.value
+
+
+def attn_strerror(status: int) -> str:
+    return lib().attn_strerror(int(status)).decode()
+
+
+def attn_version() -> int:
+    return lib().attn_version()
+
+
+# ----------------------------------------------------------------- torch helpers
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float16:
+        return ATTN_FP16
+    if t.dtype == torch.bfloat16:
+        return ATTN_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}: fp16 or bf16 only")
+
+
+def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
+            return_lse: bool = True, stream=None):
+    """Attention forward on CUDA tensors [B, H, N, d]; returns (o, lse).
+
+    ``scale`` defaults to 1/sqrt(d), the default of the pages' SDPA call
+    (YOLO11 x FlashAttention-2, kwkr.cn, section 2.2).  Inputs must be
+    contiguous (the page's transposed views need ``.contiguous()``).
+    """
+    import torch
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4:
+        raise ValueError("q, k, v must be [B, H, N, d]")
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if k.shape != (B, H, Nk, d) or v.shape != (B, H, Nk, d):
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)} k {tuple(k.shape)} v {tuple(v.shape)}")
+    if not (q.is_cuda and k.is_cuda and v.is_cuda):
+        raise ValueError("q, k, v must be CUDA tensors (no CPU path exists)")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise TypeError("q, k, v must share one dtype")
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    code = _dtype_code(q)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=q.dtype, device=q.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    st = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                  lse.data_ptr() if lse is not None else None, B, H, Nq, Nk, d, scale, causal,
+                  code, _stream_handle(stream))
+    if st != 0:
+        raise AttnError(st)
+    return out, lse
+
+
+def forward_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal=False, scale=None,
+                 stream=None):
+    """End-to-end call from (pinned) host tensors through caller-owned device buffers."""
+    B, H, Nq, d = q_h.shape
+    Nk = k_h.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    st = attn_fwd_host(q_h.data_ptr(), k_h.data_ptr(), v_h.data_ptr(), o_h.data_ptr(),
+                       lse_h.data_ptr() if lse_h is not None else None,
+                       q_d.data_ptr(), k_d.data_ptr(), v_d.data_ptr(), o_d.data_ptr(),
+                       lse_d.data_ptr() if lse_d is not None else None,
+                       B, H, Nq, Nk, d, scale, causal, _dtype_code(q_h), _stream_handle(stream))
+    if st != 0:
+        raise AttnError(st, "attn_fwd_host")

@@ -1,0 +1,320 @@
+// Host side of the attention library: argument validation, launch planning,
+// TMA tensor-map encoding, kernel launch and the C ABI declared in attn.h.
+//
+// Validation never falls back to another path: an unsupported input is an
+// error code (the pages warn that some attention kernels silently fall back
+// to a slow path for unaligned lengths -- YOLO11 x FlashAttention-2,
+// kwkr.cn, sections 4.1 and 4.2; here any length is handled by in-kernel
+// masking and anything else is rejected loudly).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "attn.h"
+#include "attn_fwd_sm100.cuh"
+
+namespace {
+
+using attn_sm100::BLOCK_M;
+using attn_sm100::BLOCK_N;
+using attn_sm100::FwdParams;
+using attn_sm100::NUM_THREADS;
+using attn_sm100::SmemLayout;
+
+constexpr int kMaxDevices = 64;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+struct DeviceInfo {
+  bool probed = false;
+  bool supported = false;
+  int sms = 0;
+  bool smem_attr[2][2] = {{false, false}, {false, false}};  // [d==128][bf16]
+};
+
+std::mutex g_dev_mutex;
+DeviceInfo g_dev[kMaxDevices];
+
+int ceil_div(long long a, long long b) { return static_cast<int>((a + b - 1) / b); }
+
+int check_args(const void* q, const void* k, const void* v, const void* o, const float* lse,
+               int B, int H, int Nq, int Nk, int d, float scale, int dtype) {
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return ATTN_ERR_NULL;
+  if (dtype != ATTN_FP16 && dtype != ATTN_BF16) return ATTN_ERR_DTYPE;
+  if (d != 64 && d != 128) return ATTN_ERR_HEAD_DIM;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return ATTN_ERR_SHAPE;
+  const long long bh = static_cast<long long>(B) * H;
+  const long long nmax = Nq > Nk ? Nq : Nk;
+  // element offsets are 64-bit; tensor-map dims must stay below 2^32; the
+  // work-unit count must fit an int
+  if (bh >= (1LL << 31) || bh * nmax * d >= (1LL << 62) ||
+      bh * ceil_div(ceil_div(Nq, BLOCK_M), 2) >= (1LL << 31))
+    return ATTN_ERR_SHAPE;
+  auto misaligned = [](const void* p, uintptr_t a) {
+    return (reinterpret_cast<uintptr_t>(p) & (a - 1)) != 0;
+  };
+  if (misaligned(q, 16) || misaligned(k, 16) || misaligned(v, 16) || misaligned(o, 16) ||
+      (lse != nullptr && misaligned(lse, 4)))
+    return ATTN_ERR_ALIGN;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_ERR_SCALE;
+  return ATTN_OK;
+}
+
+void fill_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, attn_plan_t* out) {
+  const int q_tiles = ceil_div(Nq, BLOCK_M);
+  const int q_pairs = ceil_div(q_tiles, 2);
+  const int kv_tiles = ceil_div(Nk, BLOCK_N);
+  const long long units = static_cast<long long>(B) * H * q_pairs;
+  out->num_q_tiles = q_tiles;
+  out->num_q_pairs = q_pairs;
+  out->num_kv_tiles = kv_tiles;
+  out->num_units = static_cast<int>(units);
+  out->grid = static_cast<int>(units < num_sms ? units : num_sms);
+  out->block = NUM_THREADS;
+  out->smem_bytes = d == 64 ? SmemLayout<64>::BYTES : SmemLayout<128>::BYTES;
+  out->stages = d == 64 ? SmemLayout<64>::STAGES : SmemLayout<128>::STAGES;
+  // score tiles per (batch, head): the same count the kernel's work units visit
+  long long per_head = 0;
+  for (int qt = 0; qt < q_tiles; ++qt) {
+    if (causal) {
+      const int last_row = (qt * BLOCK_M + BLOCK_M - 1 < Nq - 1) ? qt * BLOCK_M + BLOCK_M - 1 : Nq - 1;
+      const int n = last_row / BLOCK_N + 1;
+      per_head += n < kv_tiles ? n : kv_tiles;
+    } else {
+      per_head += kv_tiles;
+    }
+  }
+  out->qk_tile_products = per_head * B * H;
+}
+
+// Probe the current device once: compute capability 10.0 and SM count.
+int current_device(int* dev_out, DeviceInfo** info_out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  DeviceInfo& info = g_dev[dev];
+  if (!info.probed) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    info.supported = (major == 10 && minor == 0);
+    info.sms = sms;
+    info.probed = true;
+  }
+  if (!info.supported) return ATTN_ERR_ARCH;
+  *dev_out = dev;
+  *info_out = &info;
+  return ATTN_OK;
+}
+
+// 3-D view (d, N, B*H) of a [B, H, N, d] tensor; boxes of 64 columns x 128
+// rows with the 128-byte swizzle the tcgen05 descriptors expect.  Rows past
+// N read as zero, so ragged tails never touch the next head.
+bool encode_map(CUtensorMap* map, const void* ptr, int N, long long BH, int d, int dtype) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
+  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(BLOCK_M), 1};
+  const cuuint32_t elem_strides[3] = {1, 1, 1};
+  const CUresult r = enc(map,
+                         dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                         3, const_cast<void*>(ptr), dims, strides, box, elem_strides,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                         CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Per-thread cache of the last call's tensor maps: repeated calls on the same
+// buffers (the common case in a model loop) skip the ~µs host encode.
+struct MapCache {
+  const void* q = nullptr;
+  const void* k = nullptr;
+  const void* v = nullptr;
+  int Nq = 0, Nk = 0, d = 0, dtype = -1, dev = -1;
+  long long BH = 0;
+  CUtensorMap mq, mk, mv;
+};
+thread_local MapCache t_maps;
+
+template <int D, bool BF16>
+int launch(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo& info,
+           cudaStream_t stream) {
+  auto kernel = attn_sm100::attn_fwd_kernel<D, BF16>;
+  constexpr int smem = SmemLayout<D>::BYTES;
+  bool& attr = info.smem_attr[D == 128][BF16];
+  if (!attr) {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!attr) {
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+      }
+      attr = true;
+    }
+  }
+  kernel<<<grid, NUM_THREADS, smem, stream>>>(maps.mq, maps.mk, maps.mv, prm);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int Nq, int Nk, int d, float scale, int causal, int dtype, attn_stream_t stream) {
+  int st = check_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, dtype);
+  if (st != ATTN_OK) return st;
+  int dev = -1;
+  DeviceInfo* info = nullptr;
+  st = current_device(&dev, &info);
+  if (st != ATTN_OK) return st;
+
+  attn_plan_t plan;
+  fill_plan(B, H, Nq, Nk, d, causal, info->sms, &plan);
+  const long long BH = static_cast<long long>(B) * H;
+
+  MapCache& mc = t_maps;
+  if (mc.q != q || mc.k != k || mc.v != v || mc.Nq != Nq || mc.Nk != Nk || mc.d != d ||
+      mc.dtype != dtype || mc.dev != dev || mc.BH != BH) {
+    mc.q = nullptr;  // invalid until all three encodes succeed
+    if (!encode_map(&mc.mq, q, Nq, BH, d, dtype) || !encode_map(&mc.mk, k, Nk, BH, d, dtype) ||
+        !encode_map(&mc.mv, v, Nk, BH, d, dtype))
+      return ATTN_ERR_CUDA;
+    mc.q = q; mc.k = k; mc.v = v;
+    mc.Nq = Nq; mc.Nk = Nk; mc.d = d; mc.dtype = dtype; mc.dev = dev; mc.BH = BH;
+  }
+
+  FwdParams prm;
+  prm.o = o;
+  prm.lse = lse;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.BH = static_cast<int>(BH);
+  prm.num_q_pairs = plan.num_q_pairs;
+  prm.num_kv_tiles = plan.num_kv_tiles;
+  prm.num_units = plan.num_units;
+  prm.causal = causal ? 1 : 0;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return dtype == ATTN_BF16 ? launch<64, true>(mc, prm, plan.grid, *info, s)
+                              : launch<64, false>(mc, prm, plan.grid, *info, s);
+  return dtype == ATTN_BF16 ? launch<128, true>(mc, prm, plan.grid, *info, s)
+                            : launch<128, false>(mc, prm, plan.grid, *info, s);
+}
+
+int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                  float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                  float* lse_dev, int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                  int dtype, attn_stream_t stream) {
+  if (q_host == nullptr || k_host == nullptr || v_host == nullptr || o_host == nullptr)
+    return ATTN_ERR_NULL;
+  int st = check_args(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Nq, Nk, d, scale, dtype);
+  if (st != ATTN_OK) return st;
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t q_bytes = bh * Nq * d * 2, kv_bytes = bh * Nk * d * 2;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(k_dev, k_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(v_dev, v_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  st = attn_fwd(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Nq, Nk, d, scale, causal, dtype, stream);
+  if (st != ATTN_OK) return st;
+  if (cudaMemcpyAsync(o_host, o_dev, q_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      (lse_host != nullptr && lse_dev != nullptr &&
+       cudaMemcpyAsync(lse_host, lse_dev, bh * Nq * sizeof(float), cudaMemcpyDeviceToHost, s) !=
+           cudaSuccess)) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return ATTN_OK;
+}
+
+int attn_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, attn_plan_t* out) {
+  if (out == nullptr) return ATTN_ERR_NULL;
+  if (d != 64 && d != 128) return ATTN_ERR_HEAD_DIM;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || num_sms < 1) return ATTN_ERR_SHAPE;
+  const long long bh = static_cast<long long>(B) * H;
+  if (bh >= (1LL << 31) || bh * ceil_div(ceil_div(Nq, BLOCK_M), 2) >= (1LL << 31))
+    return ATTN_ERR_SHAPE;
+  fill_plan(B, H, Nq, Nk, d, causal, num_sms, out);
+  return ATTN_OK;
+}
+
+int attn_get_device_status(attn_stream_t stream, unsigned int* detail) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  unsigned int word = 0;
+  if (cudaMemcpyFromSymbol(&word, attn_sm100::g_attn_status, sizeof(word)) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  if (detail != nullptr) *detail = word;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpyToSymbol(attn_sm100::g_attn_status, &zero, sizeof(zero)) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    return ATTN_ERR_DEVICE_TIMEOUT;
+  }
+  return ATTN_OK;
+}
+
+const char* attn_strerror(int status) {
+  switch (status) {
+    case ATTN_OK: return "success";
+    case ATTN_ERR_NULL: return "a required pointer is NULL";
+    case ATTN_ERR_SHAPE: return "B, H, Nq and Nk must be >= 1 and the sizes must fit the index range";
+    case ATTN_ERR_HEAD_DIM: return "head dimension d must be 64 or 128";
+    case ATTN_ERR_DTYPE: return "dtype must be ATTN_FP16 or ATTN_BF16";
+    case ATTN_ERR_ALIGN: return "q, k, v, o must be 16-byte aligned and lse 4-byte aligned";
+    case ATTN_ERR_SCALE: return "scale must be finite and > 0";
+    case ATTN_ERR_ARCH: return "the current device is not compute capability 10.0 (sm_100a)";
+    case ATTN_ERR_CUDA: return "a CUDA call failed (no usable device, encode or launch error)";
+    case ATTN_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded internal wait; its output is invalid";
+    default: return "unknown status";
+  }
+}
+
+int attn_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,496 @@
+// Exact attention forward for sm_100a (B200):
+//   O = softmax(Q K^T * scale [+ top-left causal mask]) V,   lse = m + ln(l)
+//
+// The method is the tiled online softmax of the pages: "FlashAttention 深度解读"
+// (coreui.cn), section "原理" (block tiling plus online softmax kept as a
+// running max and exponent sum) and section "实现 3" (subtract the running
+// max before exponentiating); YOLO11 x FlashAttention-2 (kwkr.cn), section
+// 1.2 (rescale the accumulated output whenever a new block raises the max;
+// split work over sequence blocks, heads and batch).  The N x N score
+// matrix never leaves the SM: S lives in tensor memory (TMEM) one 128 x 128
+// tile at a time.
+//
+// Blackwell mapping (one CTA per SM, persistent over work units):
+//   * a work unit is two 128-row Q tiles of one (batch, head); the two tiles
+//     share every K/V tile the CTA loads;
+//   * warp 9 (one lane) issues TMA loads: the unit's two Q tiles, then K_j and
+//     V_j for j = 0..n-1 into a ring of STAGES shared-memory slots, each slot
+//     guarded by a full / empty mbarrier pair;
+//   * warp 8 (one lane) issues tcgen05.mma: S_t = Q_t K_j^T into TMEM (fp32),
+//     and O_t += P_t V_j with P_t read from TMEM (it overwrites S_t, packed
+//     as 16-bit pairs); tcgen05.commit signals the softmax warps and releases
+//     ring slots;
+//   * warps 0-3 own Q tile 0 and warps 4-7 own Q tile 1: one thread per
+//     query row reads its S row from TMEM, masks, updates the running max
+//     m (base-2, pre-multiplied by scale*log2 e) and sum l, writes P, and
+//     rescales its O row in TMEM by 2^(m_old - m_new) when the max rose.
+//     While one warpgroup runs its softmax the tensor core works on the
+//     other tile, so exp and MMA overlap.
+//   * the epilogue divides O by l, rounds to the input dtype and stores the
+//     rows below Nq; lse = (m + log2 l) * ln 2.
+//
+// Every mbarrier wait is bounded (about one second of %globaltimer); on
+// timeout the kernel records where in a device status word, tells the other
+// roles to stop, waits (bounded) for its own TMA loads and MMAs to land,
+// frees TMEM and returns.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+
+#include "sm100_ptx.cuh"
+
+namespace attn_sm100 {
+
+constexpr int BLOCK_M = 128;     // query rows per Q tile (= TMEM lanes)
+constexpr int BLOCK_N = 128;     // keys per K / V tile
+constexpr int NUM_THREADS = 320; // 8 softmax warps + MMA warp + load warp
+constexpr int MMA_WARP = 8;
+constexpr int LOAD_WARP = 9;
+constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
+
+// Device status word: 0 = healthy; otherwise 0x80000000 | site.
+__device__ unsigned int g_attn_status = 0;
+
+enum WaitSite : uint32_t {
+  SITE_LOAD_Q_EMPTY = 1,
+  SITE_LOAD_KV_EMPTY = 2,
+  SITE_MMA_Q_FULL = 3,
+  SITE_MMA_KV_FULL = 4,
+  SITE_MMA_P_FULL = 5,
+  SITE_SOFTMAX_S_FULL = 6,
+  SITE_SOFTMAX_O_FULL = 7,
+  SITE_DRAIN = 8,
+};
+
+struct FwdParams {
+  void* o;         // [B, H, Nq, D] fp16 / bf16
+  float* lse;      // [B, H, Nq] fp32, or nullptr
+  int Nq, Nk, BH;
+  int num_q_pairs;  // ceil(ceil(Nq / 128) / 2)
+  int num_kv_tiles; // ceil(Nk / 128)
+  int num_units;    // BH * num_q_pairs
+  int causal;
+  float scale_log2; // scale * log2(e)
+};
+
+template <int D>
+struct SmemLayout {
+  static constexpr int HALF_BYTES = BLOCK_M * 64 * 2;  // one 64-column, 128-byte-swizzled slab
+  static constexpr int HALVES = D / 64;
+  static constexpr int TILE_BYTES = HALVES * HALF_BYTES;
+  static constexpr int STAGES = (D == 64) ? 8 : 4;
+  static constexpr int Q_OFF = 0;
+  static constexpr int KV_OFF = Q_OFF + 2 * TILE_BYTES;
+  static constexpr int BAR_OFF = KV_OFF + STAGES * TILE_BYTES;
+  // mbarrier indices
+  static constexpr int KV_FULL = 0;
+  static constexpr int KV_EMPTY = STAGES;
+  static constexpr int Q_FULL = 2 * STAGES;
+  static constexpr int Q_EMPTY = 2 * STAGES + 1;
+  static constexpr int S_FULL = 2 * STAGES + 2;  // + tile
+  static constexpr int P_FULL = 2 * STAGES + 4;  // + tile
+  static constexpr int O_FULL = 2 * STAGES + 6;  // + tile
+  static constexpr int DRAIN = 2 * STAGES + 8;
+  static constexpr int NUM_BARS = 2 * STAGES + 9;
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // TMEM address, abort flag
+  static constexpr int BYTES = MISC_OFF + 16 + 1024;      // + slack to align the base to 1 KB
+  // TMEM columns (512 allocated): S/P of tile 0 and 1, then O of tile 0 and 1
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t S_COL = 0;    // + 128 * tile
+  static constexpr uint32_t O_COL = 256;  // + D * tile
+};
+
+struct Unit {
+  int bh;
+  int q0;    // first query row of tile 0
+  int n[2];  // K/V tiles each Q tile visits (0 = tile lies past Nq)
+  int nmax;
+};
+
+// Work-unit order.  Causal: heaviest Q pairs first (longest-processing-time
+// order) so the persistent CTAs finish together.  Non-causal: the Q pairs of
+// one head are adjacent, so CTAs running at the same time share that head's
+// K/V through L2.
+__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
+  Unit w;
+  int qp;
+  if (p.causal) {
+    qp = p.num_q_pairs - 1 - u / p.BH;
+    w.bh = u % p.BH;
+  } else {
+    w.bh = u / p.num_q_pairs;
+    qp = u % p.num_q_pairs;
+  }
+  w.q0 = qp * 2 * BLOCK_M;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int qs = w.q0 + t * BLOCK_M;
+    int n;
+    if (qs >= p.Nq) {
+      n = 0;
+    } else if (p.causal) {
+      const int last_row = min(qs + BLOCK_M - 1, p.Nq - 1);
+      n = min(p.num_kv_tiles, last_row / BLOCK_N + 1);
+    } else {
+      n = p.num_kv_tiles;
+    }
+    w.n[t] = n;
+  }
+  w.nmax = max(w.n[0], w.n[1]);
+  return w;
+}
+
+// Bounded wait on one mbarrier phase.  Returns false on timeout (status word
+// set, abort flag raised) or, when honour_abort, once another role aborted.
+__device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                        uint32_t site, bool honour_abort) {
+  const uint64_t t0 = global_timer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int i = 0; i < 128; ++i) {
+      if (mbar_try_wait(bar, parity)) return true;
+    }
+    if (honour_abort && *abort_flag) return false;
+    if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
+      atomicCAS(&g_attn_status, 0u, 0x80000000u | site);
+      *abort_flag = 1;
+      return false;
+    }
+  }
+}
+
+__device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return wait_phase(bar, parity, abort_flag, site, true);
+}
+
+template <int D, bool BF16>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using L = SmemLayout<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_addr(smem);
+  const int warp = threadIdx.x / 32;
+  const int lane = threadIdx.x % 32;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
+  auto bar = [&](int i) -> uint32_t { return sbase + L::BAR_OFF + 8u * i; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L::STAGES; ++s) {
+      mbar_init(bar(L::KV_FULL + s), 1);
+      mbar_init(bar(L::KV_EMPTY + s), 1);
+    }
+    mbar_init(bar(L::Q_FULL), 1);
+    mbar_init(bar(L::Q_EMPTY), 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(L::S_FULL + t), 1);
+      mbar_init(bar(L::P_FULL + t), 4 * 32);
+      mbar_init(bar(L::O_FULL + t), 1);
+    }
+    mbar_init(bar(L::DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbarrier_init();
+  }
+  if (warp == LOAD_WARP && lane == 0) {
+    prefetch_tensormap(&tm_q);
+    prefetch_tensormap(&tm_k);
+    prefetch_tensormap(&tm_v);
+  }
+  if (warp == MMA_WARP) {
+    tmem_alloc(smem_addr(tmem_slot), L::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == LOAD_WARP) {
+    // ------------------------------------------------------------- TMA producer
+    if (lane == 0) {
+      const uint32_t q_smem = sbase + L::Q_OFF;
+      const uint32_t kv_smem = sbase + L::KV_OFF;
+      uint32_t kv_it = 0, units = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        const Unit w = decode_unit(p, u);
+        if (units > 0) {
+          ok = wait_fast(bar(L::Q_EMPTY), (units - 1) & 1, abort_flag, SITE_LOAD_Q_EMPTY);
+          if (!ok) break;
+        }
+        mbar_arrive_expect_tx(bar(L::Q_FULL), 2 * L::TILE_BYTES);
+        for (int t = 0; t < 2; ++t)
+          for (int h = 0; h < L::HALVES; ++h)
+            tma_load_3d(q_smem + t * L::TILE_BYTES + h * L::HALF_BYTES, &tm_q, bar(L::Q_FULL),
+                        h * 64, w.q0 + t * BLOCK_M, w.bh);
+        ++units;
+        for (int j = 0; ok && j < w.nmax; ++j) {
+          for (int which = 0; which < 2; ++which) {
+            const uint32_t st = kv_it % L::STAGES;
+            const uint32_t ph = (kv_it / L::STAGES) & 1;
+            if (kv_it >= static_cast<uint32_t>(L::STAGES)) {
+              ok = wait_fast(bar(L::KV_EMPTY + st), ph ^ 1, abort_flag, SITE_LOAD_KV_EMPTY);
+              if (!ok) break;
+            }
+            mbar_arrive_expect_tx(bar(L::KV_FULL + st), L::TILE_BYTES);
+            for (int h = 0; h < L::HALVES; ++h)
+              tma_load_3d(kv_smem + st * L::TILE_BYTES + h * L::HALF_BYTES, which ? &tm_v : &tm_k,
+                          bar(L::KV_FULL + st), h * 64, j * BLOCK_N, w.bh);
+            ++kv_it;
+          }
+        }
+      }
+      // Every issued load must have landed before the CTA may exit.
+      const uint32_t first = kv_it > static_cast<uint32_t>(L::STAGES) ? kv_it - L::STAGES : 0;
+      for (uint32_t i = first; i < kv_it; ++i)
+        wait_phase(bar(L::KV_FULL + i % L::STAGES), (i / L::STAGES) & 1, abort_flag, SITE_DRAIN,
+                   false);
+      if (units > 0) wait_phase(bar(L::Q_FULL), (units - 1) & 1, abort_flag, SITE_DRAIN, false);
+    }
+    __syncwarp();
+  } else if (warp == MMA_WARP) {
+    // ------------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_f16(BF16, false, false, BLOCK_M, BLOCK_N);
+      constexpr uint32_t IDESC_O = idesc_f16(BF16, false, true, BLOCK_M, D);
+      const uint32_t q_smem = sbase + L::Q_OFF;
+      const uint32_t kv_smem = sbase + L::KV_OFF;
+
+      // S_t = Q_t K^T: both operands K-major (head dim contiguous), 128-byte
+      // swizzle, 8-row groups 1024 bytes apart; each k-step covers 16
+      // elements = 32 bytes of a 128-byte row, the head dim > 64 continues in
+      // the next 16 KB slab.
+      auto issue_s = [&](int t, uint32_t stage) {
+        const uint32_t qa = q_smem + t * L::TILE_BYTES;
+        const uint32_t ka = kv_smem + stage * L::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk / 4) * L::HALF_BYTES + (kk % 4) * 32;
+          mma_ss(tmem_base + L::S_COL + 128 * t, sw128_desc(qa + off, 16, 1024),
+                 sw128_desc(ka + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_t += P_t V: P from TMEM (16 keys = 8 columns per k-step), V
+      // MN-major (head dim contiguous): 8-key groups 1024 bytes apart,
+      // 64-column slabs 16 KB apart; each k-step advances 16 keys = 2 KB.
+      auto issue_pv = [&](int t, uint32_t stage, bool accumulate) {
+        const uint32_t va = kv_smem + stage * L::TILE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
+          mma_ts(tmem_base + L::O_COL + D * t, tmem_base + L::S_COL + 128 * t + kk * 8,
+                 sw128_desc(va + kk * 2048, L::HALF_BYTES, 1024), IDESC_O,
+                 (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      uint32_t kv_it = 0, q_phase = 0;
+      uint32_t p_phase[2] = {0, 0};
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+        const Unit w = decode_unit(p, u);
+        ok = wait_fast(bar(L::Q_FULL), q_phase, abort_flag, SITE_MMA_Q_FULL);
+        if (!ok) break;
+        q_phase ^= 1;
+        {
+          const uint32_t st = kv_it % L::STAGES, ph = (kv_it / L::STAGES) & 1;
+          ++kv_it;
+          ok = wait_fast(bar(L::KV_FULL + st), ph, abort_flag, SITE_MMA_KV_FULL);
+          if (!ok) break;
+          tc_fence_after();
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (w.n[t] > 0) {
+              issue_s(t, st);
+              mma_commit(bar(L::S_FULL + t));
+            }
+          }
+          mma_commit(bar(L::KV_EMPTY + st));
+        }
+        for (int j = 0; ok && j < w.nmax; ++j) {
+          const uint32_t vst = kv_it % L::STAGES, vph = (kv_it / L::STAGES) & 1;
+          ++kv_it;
+          const bool has_next = j + 1 < w.nmax;
+          uint32_t kst = 0, kph = 0;
+          if (has_next) {
+            kst = kv_it % L::STAGES;
+            kph = (kv_it / L::STAGES) & 1;
+            ++kv_it;
+          }
+          ok = wait_fast(bar(L::KV_FULL + vst), vph, abort_flag, SITE_MMA_KV_FULL);
+          if (!ok) break;
+          bool k_ready = false;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            if (!ok || j >= w.n[t]) continue;
+            ok = wait_fast(bar(L::P_FULL + t), p_phase[t], abort_flag, SITE_MMA_P_FULL);
+            if (!ok) continue;
+            p_phase[t] ^= 1;
+            tc_fence_after();
+            issue_pv(t, vst, j > 0);
+            if (j + 1 < w.n[t]) {
+              if (!k_ready) {
+                ok = wait_fast(bar(L::KV_FULL + kst), kph, abort_flag, SITE_MMA_KV_FULL);
+                if (!ok) continue;
+                tc_fence_after();
+                k_ready = true;
+              }
+              issue_s(t, kst);
+              mma_commit(bar(L::S_FULL + t));
+            } else {
+              mma_commit(bar(L::O_FULL + t));
+            }
+          }
+          if (!ok) break;
+          mma_commit(bar(L::KV_EMPTY + vst));
+          if (has_next) {
+            if (!k_ready) {
+              ok = wait_fast(bar(L::KV_FULL + kst), kph, abort_flag, SITE_MMA_KV_FULL);
+              if (!ok) break;
+            }
+            mma_commit(bar(L::KV_EMPTY + kst));
+          }
+        }
+        if (!ok) break;
+        mma_commit(bar(L::Q_EMPTY));
+      }
+      // All MMAs (and their commits) must be finished before TMEM is freed.
+      mma_commit(bar(L::DRAIN));
+      wait_phase(bar(L::DRAIN), 0, abort_flag, SITE_DRAIN, false);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------- softmax
+    const int t = warp / 4;
+    const int quarter = warp % 4;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t tS = tmem_base + lane_off + L::S_COL + 128 * t;
+    const uint32_t tO = tmem_base + lane_off + L::O_COL + D * t;
+    const float sl2 = p.scale_log2;
+    uint32_t s_phase = 0, o_phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
+      const Unit w = decode_unit(p, u);
+      const int n = t ? w.n[1] : w.n[0];
+      if (n == 0) continue;
+      const int q_start = w.q0 + t * BLOCK_M;
+      const int row = q_start + r;
+      // last key this row may see (top-left causal: key j <= query i)
+      const int last_key = p.causal ? min(p.Nk - 1, row) : (p.Nk - 1);
+      float m = -INFINITY, l = 0.f;
+      for (int j = 0; j < n; ++j) {
+        ok = wait_fast(bar(L::S_FULL + t), s_phase, abort_flag, SITE_SOFTMAX_S_FULL);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        s_phase ^= 1;
+        tc_fence_after();
+        uint32_t sr[128];
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * c));
+        tmem_wait_ld();
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+
+        const int k0 = j * BLOCK_N;
+        const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > q_start);
+        if (need_mask) {
+          const int lim = last_key - k0;  // columns > lim are masked
+#pragma unroll
+          for (int c = 0; c < 128; ++c) s[c] = (c > lim) ? -INFINITY : s[c];
+        }
+        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+#pragma unroll
+        for (int c = 4; c < 128; c += 4) {
+          mx0 = fmaxf(mx0, s[c]);
+          mx1 = fmaxf(mx1, s[c + 1]);
+          mx2 = fmaxf(mx2, s[c + 2]);
+          mx3 = fmaxf(mx3, s[c + 3]);
+        }
+        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float m_new = fmaxf(m, mx * sl2);
+        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+        const float alpha = ex2_approx(m - m_use);
+        const float neg_m = -m_use;
+
+        float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+        for (int hblk = 0; hblk < 2; ++hblk) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float a = ex2_approx(fmaf(s[64 * hblk + 2 * c], sl2, neg_m));
+            const float b = ex2_approx(fmaf(s[64 * hblk + 2 * c + 1], sl2, neg_m));
+            sum0 += a;
+            sum1 += b;
+            pk[c] = pack2<BF16>(a, b);
+          }
+          tmem_st32(tS + 32 * hblk, pk);
+        }
+        l = l * alpha + (sum0 + sum1);
+        m = m_new;
+
+        if (j > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
+#pragma unroll
+          for (int c0 = 0; c0 < D; c0 += 32) {
+            uint32_t o[32];
+            tmem_ld32(tO + c0, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tO + c0, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(L::P_FULL + t));
+      }
+      if (!ok) break;
+
+      // ----------------------------------------------------------- epilogue
+      ok = wait_fast(bar(L::O_FULL + t), o_phase, abort_flag, SITE_SOFTMAX_O_FULL);
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) break;
+      o_phase ^= 1;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const bool in_range = row < p.Nq;
+      uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
+                                             (static_cast<size_t>(w.bh) * p.Nq + row) * D);
+#pragma unroll
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        tmem_ld32(tO + c0, o);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i)
+          pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+        if (in_range) {
+#pragma unroll
+          for (int v4 = 0; v4 < 4; ++v4)
+            orow[c0 / 8 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+        }
+      }
+      if (p.lse != nullptr && in_range)
+        p.lse[static_cast<size_t>(w.bh) * p.Nq + row] = (m + lg2_approx(l)) * 0.69314718055994531f;
+      tc_fence_before();
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == MMA_WARP) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+}
+
+}  // namespace attn_sm100

@@ -1,0 +1,137 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) exact attention forward.
+ *
+ *   O = softmax(Q K^T * scale [+ causal mask]) V,    lse = logsumexp of the scaled scores
+ *
+ * The operation is the attention formula of "FlashAttention 深度解读：让大模型注意力机制
+ * 一口气算完" (coreui.cn), section "背景", computed by the tiled online softmax of its section
+ * "原理" and of the YOLO11 x FlashAttention-2 page (kwkr.cn), section 1.2: the N x N score
+ * matrix never reaches HBM.  The argument list mirrors the pages' Python entry points,
+ * torch's scaled_dot_product_attention(q, k, v, is_causal, scale) (kwkr.cn, section 2.2) and
+ * flash_attention(q, k, v, causal) (coreui.cn, section "怎么用"); dropout is not supported
+ * (inference, dropout_p = 0).
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are contiguous row-major.  q is [B, H, Nq, d]; k and v are [B, H, Nk, d];
+ *     o is [B, H, Nq, d], all in `dtype` (ATTN_FP16 or ATTN_BF16).  lse is [B, H, Nq]
+ *     float32, natural log: lse[i] = ln(sum_j exp(scale * q_i . k_j)) over the visible keys.
+ *   - causal != 0 applies the top-left aligned mask: query i sees key j iff j <= i (the
+ *     convention of torch's is_causal).  Every query row sees at least key 0.
+ *   - scale is the factor applied to Q K^T; the usual value is 1/sqrt(d).
+ *   - All memory is owned by the caller.  The library allocates nothing per call.
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; 0 = legacy default stream).  A
+ *     return of ATTN_OK means the arguments were valid and the kernel was enqueued.
+ *   - No fallback path exists: an unsupported input returns an error code; nothing is
+ *     computed a different way.
+ *   - Thread safety: calls from several host threads are safe.
+ */
+#ifndef ATTN_SM100_ATTN_H_
+#define ATTN_SM100_ATTN_H_
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* attn_stream_t;
+
+typedef enum {
+  ATTN_FP16 = 0,
+  ATTN_BF16 = 1
+} attn_dtype_t;
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_ERR_NULL = 1,           /* a required pointer is NULL */
+  ATTN_ERR_SHAPE = 2,          /* B, H, Nq or Nk < 1, or the sizes overflow the index range */
+  ATTN_ERR_HEAD_DIM = 3,       /* d is not 64 or 128 */
+  ATTN_ERR_DTYPE = 4,          /* dtype is not ATTN_FP16 / ATTN_BF16 */
+  ATTN_ERR_ALIGN = 5,          /* q, k, v, o not 16-byte aligned, or lse not 4-byte aligned */
+  ATTN_ERR_SCALE = 6,          /* scale is not finite and > 0 */
+  ATTN_ERR_ARCH = 7,           /* current device is not compute capability 10.0 (B200) */
+  ATTN_ERR_CUDA = 8,           /* a CUDA runtime / driver call failed (no device, launch error) */
+  ATTN_ERR_DEVICE_TIMEOUT = 9  /* a kernel gave up waiting (see attn_get_device_status) */
+} attn_status_t;
+
+/* Launch geometry for one call (see attn_plan). */
+typedef struct {
+  int num_q_tiles;   /* ceil(Nq / 128): 128-row query tiles per (batch, head)            */
+  int num_q_pairs;   /* ceil(num_q_tiles / 2): a work unit is two query tiles             */
+  int num_kv_tiles;  /* ceil(Nk / 128): 128-key tiles per (batch, head)                   */
+  int num_units;     /* B * H * num_q_pairs work units                                    */
+  int grid;          /* persistent CTAs launched: min(num_units, SM count)                */
+  int block;         /* threads per CTA                                                   */
+  int smem_bytes;    /* dynamic shared memory per CTA                                     */
+  int stages;        /* K/V shared-memory ring slots                                      */
+  long long qk_tile_products; /* 128x128 score tiles computed (incl. masked tail tiles)   */
+} attn_plan_t;
+
+/*
+ * attn_fwd -- the attention forward on device memory.
+ *
+ *   q, k, v  device pointers, 16-byte aligned, layouts above, read only.
+ *   o        device pointer, 16-byte aligned, [B, H, Nq, d], written (rows < Nq only).
+ *   lse      device pointer to [B, H, Nq] float32, 4-byte aligned, written; or NULL to skip.
+ *   B, H     batch and heads, >= 1.    Nq, Nk  query and key counts, >= 1 (any value; no
+ *            multiple-of-8 or multiple-of-128 requirement -- ragged tails are masked in the
+ *            kernel).
+ *   d        head dimension, 64 or 128.
+ *   scale    softmax scale, finite and > 0.
+ *   causal   0 = full attention, nonzero = top-left causal mask.
+ *   dtype    ATTN_FP16 or ATTN_BF16 (q, k, v and o share it).
+ *   stream   CUDA stream to enqueue on.
+ *
+ * Returns ATTN_OK after enqueueing.  Argument errors are detected on the host before any
+ * CUDA call, in this order: ATTN_ERR_NULL, ATTN_ERR_DTYPE, ATTN_ERR_HEAD_DIM, ATTN_ERR_SHAPE,
+ * ATTN_ERR_ALIGN, ATTN_ERR_SCALE; then ATTN_ERR_CUDA (no usable device) or ATTN_ERR_ARCH.
+ * On any error nothing is enqueued and o / lse are untouched.  Precision: fp32 accumulation
+ * and softmax statistics; P is rounded to `dtype` before the P V product; O is rounded to
+ * nearest-even once.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int Nq, int Nk, int d, float scale, int causal, int dtype, attn_stream_t stream);
+
+/*
+ * attn_fwd_host -- the same forward, end to end from host memory.
+ *
+ * Enqueues on `stream`: host->device copies of q_host, k_host, v_host into the caller's
+ * device buffers q_dev, k_dev, v_dev; attn_fwd on them into o_dev / lse_dev; device->host
+ * copies of o_dev into o_host and (when both lse pointers are non-NULL) lse_dev into
+ * lse_host.  Host buffers should be pinned (cudaHostAlloc / cudaHostRegister) for the copies
+ * to be asynchronous.  The caller synchronises `stream` before reading o_host.  Argument
+ * rules and error codes are those of attn_fwd; every host and device pointer except the lse
+ * pair must be non-NULL.  Nothing is allocated.
+ */
+int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
+                  float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
+                  float* lse_dev, int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                  int dtype, attn_stream_t stream);
+
+/*
+ * attn_plan -- the launch geometry attn_fwd would use for these sizes on a GPU with
+ * `num_sms` SMs (pure host arithmetic; needs no GPU).  Returns ATTN_ERR_SHAPE /
+ * ATTN_ERR_HEAD_DIM / ATTN_ERR_NULL on bad arguments, else ATTN_OK with *out filled.
+ */
+int attn_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, attn_plan_t* out);
+
+/*
+ * attn_get_device_status -- synchronises `stream`, then reads and clears the device status
+ * word the kernels write when a bounded internal wait gives up (about one second).  Returns
+ * ATTN_OK when healthy, ATTN_ERR_DEVICE_TIMEOUT when a kernel timed out (the result of that
+ * call is invalid; the CUDA context stays usable), ATTN_ERR_CUDA if the synchronisation or
+ * the read fails.  When `detail` is non-NULL it receives the raw status word (0 = healthy;
+ * else 0x80000000 | wait site).
+ */
+int attn_get_device_status(attn_stream_t stream, unsigned int* detail);
+
+/* Static English message for a status code; never NULL. */
+const char* attn_strerror(int status);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int attn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_SM100_ATTN_H_ */

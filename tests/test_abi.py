@@ -1,0 +1,146 @@
+"""Host-side tests of the C ABI (no GPU needed).
+
+* the library loads and exports every function ``include/attn.h`` declares;
+* argument validation returns the documented code before any CUDA call;
+* ``attn_plan`` gives the launch geometry the kernel uses;
+* without a usable device a valid call fails loudly (ATTN_ERR_CUDA) -- there
+  is no CPU fallback.
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import exact_attention_153_b200 as A
+from exact_attention_153_b200 import build_lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn.h")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build_lib.build()
+
+
+def header_functions():
+    text = open(HEADER, encoding="utf-8").read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(attn_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    assert header_functions() == sorted([
+        "attn_fwd", "attn_fwd_host", "attn_plan", "attn_get_device_status", "attn_strerror",
+        "attn_version"])
+
+
+def test_every_declared_symbol_is_exported():
+    lib = ctypes.CDLL(A.library_path())
+    for name in header_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", A.library_path()], capture_output=True,
+                         text=True).stdout
+    exported = set(re.findall(r"\bT (attn_\w+)", out))
+    assert set(header_functions()) <= exported
+
+
+def test_status_enum_matches_header():
+    text = open(HEADER, encoding="utf-8").read()
+    for code, name in A.STATUS_NAMES.items():
+        assert re.search(rf"\b{name}\s*=\s*{code}\b", text), name
+
+
+def test_strerror_and_version():
+    for code in range(10):
+        assert A.attn_strerror(code)
+    assert A.attn_strerror(1234) == "unknown status"
+    assert A.attn_version() == 100
+
+
+GOOD = dict(q=0x10000, k=0x20000, v=0x30000, o=0x40000, lse=0x50000, B=1, H=2, Nq=400, Nk=400,
+            d=64, scale=0.125, causal=0, dtype=A.ATTN_FP16, stream=None)
+
+
+def call(**kw):
+    a = dict(GOOD)
+    a.update(kw)
+    return A.attn_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["H"], a["Nq"], a["Nk"],
+                      a["d"], a["scale"], a["causal"], a["dtype"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(k=None), 1), (dict(v=None), 1), (dict(o=None), 1),
+    (dict(dtype=2), 4), (dict(dtype=-1), 4),
+    (dict(d=32), 3), (dict(d=96), 3), (dict(d=256), 3),
+    (dict(B=0), 2), (dict(H=0), 2), (dict(Nq=0), 2), (dict(Nk=0), 2), (dict(Nk=-5), 2),
+    (dict(B=1 << 16, H=1 << 15), 2),
+    (dict(q=0x10008), 5), (dict(o=0x40004), 5), (dict(lse=0x50002), 5),
+    (dict(scale=0.0), 6), (dict(scale=-1.0), 6), (dict(scale=float("nan")), 6),
+    (dict(scale=float("inf")), 6),
+])
+def test_argument_errors(kw, code):
+    assert call(**kw) == code
+
+
+def test_error_order_null_first():
+    assert call(q=None, d=7, dtype=9) == 1
+    assert call(dtype=9, d=7) == 4
+    assert call(d=7, B=0) == 3
+
+
+def test_lse_may_be_null():
+    # With valid arguments the next step needs a device; this host has none
+    # (or it is not an sm_100 part): the call must fail, not compute elsewhere.
+    st = call(lse=None)
+    assert st in (0, 7, 8)
+
+
+def test_no_silent_fallback_without_device():
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present; covered by the gpu tests")
+    assert call() == 8
+    assert A.attn_get_device_status(0)[0] == 8
+
+
+def test_host_entry_argument_errors():
+    base = [0x1000] * 10
+    args = dict(B=1, H=1, Nq=8, Nk=8, d=64, scale=0.125, causal=0, dtype=0, stream=None)
+    assert A.attn_fwd_host(None, *base[1:], *args.values()) == 1
+    ptrs = list(base)
+    ptrs[5] = None  # q_dev
+    assert A.attn_fwd_host(*ptrs, *args.values()) == 1
+    args["d"] = 80
+    assert A.attn_fwd_host(*base, *args.values()) == 3
+
+
+def test_plan_geometry():
+    p = A.attn_plan(1, 2, 400, 400, 64, 0, 148)
+    assert (p["num_q_tiles"], p["num_q_pairs"], p["num_kv_tiles"], p["num_units"]) == (4, 2, 4, 4)
+    assert p["grid"] == 4 and p["block"] == 320
+    assert p["qk_tile_products"] == 2 * 4 * 4
+    p = A.attn_plan(16, 4, 1600, 1600, 64, 0, 148)
+    assert (p["num_q_tiles"], p["num_q_pairs"], p["num_units"], p["grid"]) == (13, 7, 448, 148)
+    assert p["smem_bytes"] <= 232448
+    p = A.attn_plan(32, 16, 2048, 2048, 64, 1, 148)
+    # causal: query tile i visits key tiles 0..i
+    assert p["qk_tile_products"] == 32 * 16 * sum(range(1, 17))
+    p = A.attn_plan(1, 32, 32768, 32768, 128, 1, 148)
+    assert p["stages"] == 4 and p["smem_bytes"] <= 232448
+    assert p["qk_tile_products"] == 32 * sum(range(1, 257))
+    # ragged causal with Nq != Nk (top-left): rows past Nk see every key
+    p = A.attn_plan(1, 1, 300, 200, 64, 1, 148)
+    assert p["qk_tile_products"] == 1 + 2 + 2
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=48), 3), (dict(B=0), 2), (dict(num_sms=0), 2)])
+def test_plan_errors(kw, code):
+    a = dict(B=1, H=1, Nq=10, Nk=10, d=64, causal=0, num_sms=148)
+    a.update(kw)
+    with pytest.raises(A.AttnError) as e:
+        A.attn_plan(*a.values())
+    assert e.value.status == code

@@ -1,0 +1,251 @@
+"""GPU parity: the sm_100a kernel against the float64 CPU oracle.
+
+Bar (fixed for every case): max |O_gpu - O_oracle| <= 4e-3 for fp16 and 2e-2
+for bf16; max |lse_gpu - lse_oracle| <= 1e-3.  Inputs are the seeded
+workloads; the oracle sees exactly the fp16 / bf16 values the GPU sees.
+Small shapes compare every element; the full-size workloads compare sampled
+rows (each computed by the oracle against the full K and V) and check that
+every output element is finite and that nothing outside O and lse is
+written.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import exact_attention_153_b200 as A
+import oracle
+from exact_attention_153_b200 import build_lib
+from seeded_inputs import WORKLOADS, make_qkv, make_workload_qkv
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"fp16": 4e-3, "bf16": 2e-2}
+LSE_TOL = 1e-3
+SENTINEL = 0x7E01  # a NaN pattern in fp16 and bf16 alike; the kernel never writes it
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build_lib.build()
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+
+
+def _run(q, k, v, causal, scale):
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o, lse = A.forward(qd, kd, vd, causal=causal, scale=scale)
+    torch.cuda.synchronize()
+    st, word = A.attn_get_device_status()
+    assert st == 0, f"device status {word:#x}"
+    return o.cpu(), lse.cpu()
+
+
+def _err(a, b):
+    return float(np.max(np.abs(np.asarray(a, np.float64) - np.asarray(b, np.float64))))
+
+
+def _check_full(q, k, v, causal, scale, dtype):
+    o, lse = _run(q, k, v, causal, scale)
+    o_ref, lse_ref = oracle.attention_f64(q, k, v, scale, causal)
+    eo = _err(o.double().numpy(), o_ref)
+    el = _err(lse.double().numpy(), lse_ref)
+    assert eo <= TOL[dtype], f"O err {eo:.3e}"
+    assert el <= LSE_TOL, f"lse err {el:.3e}"
+    return eo, el
+
+
+SQUARE = [1, 7, 127, 128, 129, 255, 256, 257, 400, 1000]
+
+
+@pytest.mark.parametrize("N", SQUARE)
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_square_shapes(N, d, dtype, causal):
+    q, k, v = make_qkv(2, 3, N, N, d, dtype, seed=N * 10 + d + (dtype == "bf16"))
+    _check_full(q, k, v, causal, 1.0 / math.sqrt(d), dtype)
+
+
+@pytest.mark.parametrize("Nq,Nk", [(100, 300), (300, 100), (513, 129), (1, 1000), (1000, 1),
+                                   (129, 700), (640, 257)])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_rectangular_shapes(Nq, Nk, d, causal):
+    dtype = "fp16" if d == 64 else "bf16"
+    q, k, v = make_qkv(1, 2, Nq, Nk, d, dtype, seed=Nq + 7 * Nk + d)
+    _check_full(q, k, v, causal, 1.0 / math.sqrt(d), dtype)
+
+
+@pytest.mark.parametrize("scale", [0.01, 0.3, 1.0])
+def test_other_scales(scale):
+    q, k, v = make_qkv(1, 2, 300, 300, 64, "fp16", seed=5)
+    _check_full(q, k, v, True, scale, "fp16")
+
+
+def test_many_units_persistent_loop():
+    """More work units than SMs: every CTA loops over several units."""
+    q, k, v = make_qkv(8, 40, 257, 257, 64, "bf16", seed=11)
+    _check_full(q, k, v, True, 0.125, "bf16")
+    _check_full(q, k, v, False, 0.125, "bf16")
+
+
+# ------------------------------------------------------------ the five workloads
+
+@pytest.mark.parametrize("idx", [0, 1])
+def test_workload_full_compare(idx):
+    w = WORKLOADS[idx]
+    q, k, v = make_workload_qkv(w)
+    _check_full(q, k, v, w.causal, w.scale, w.dtype)
+
+
+def _sample_rows(N, rng, extra=24):
+    fixed = [0, 1, 2, 126, 127, 128, 129, N // 2, N - 129, N - 128, N - 2, N - 1]
+    rows = set(r for r in fixed if 0 <= r < N)
+    rows.update(rng.integers(0, N, size=extra).tolist())
+    return np.array(sorted(rows))
+
+
+@pytest.mark.parametrize("idx", [2, 3, 4])
+def test_workload_sampled_rows(idx):
+    w = WORKLOADS[idx]
+    q, k, v = make_workload_qkv(w)
+    o, lse = _run(q, k, v, w.causal, w.scale)
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    rng = np.random.default_rng(w.seed)
+    heads = sorted(set([(0, 0), (w.B - 1, w.H - 1)] +
+                       [(int(rng.integers(w.B)), int(rng.integers(w.H))) for _ in range(3)]))
+    worst_o = worst_l = 0.0
+    for b, h in heads:
+        rows = _sample_rows(w.Nq, rng)
+        o_ref, l_ref = oracle.attention_head_rows(q[b, h, rows], k[b, h], v[b, h], w.scale,
+                                                  w.causal, rows)
+        worst_o = max(worst_o, _err(o[b, h, rows].double().numpy(), o_ref))
+        worst_l = max(worst_l, _err(lse[b, h, rows].double().numpy(), l_ref))
+    assert worst_o <= TOL[w.dtype], f"O err {worst_o:.3e}"
+    assert worst_l <= LSE_TOL, f"lse err {worst_l:.3e}"
+
+
+# ------------------------------------------------------------ invariants on the GPU
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_v(causal):
+    q, k, _ = make_qkv(2, 2, 300, 300, 64, "fp16", seed=21)
+    r = torch.randn(64, generator=torch.Generator().manual_seed(3)).half()
+    v = r.expand(2, 2, 300, 64).contiguous()
+    o, _ = _run(q, k, v, causal, 0.125)
+    assert _err(o.double().numpy(), np.broadcast_to(r.double().numpy(), o.shape)) <= TOL["fp16"]
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_q_zero_closed_form(causal, d):
+    N = 333
+    _, k, v = make_qkv(1, 2, N, N, d, "bf16", seed=22)
+    q = torch.zeros(1, 2, N, d, dtype=torch.bfloat16)
+    o, lse = _run(q, k, v, causal, 1.0 / math.sqrt(d))
+    vf = v.double().numpy()
+    if causal:
+        mean = np.cumsum(vf, axis=2) / np.arange(1, N + 1)[None, None, :, None]
+        lse_ref = np.broadcast_to(np.log(np.arange(1, N + 1)), (1, 2, N))
+    else:
+        mean = np.broadcast_to(vf.mean(axis=2, keepdims=True), vf.shape)
+        lse_ref = np.full((1, 2, N), math.log(N))
+    assert _err(o.double().numpy(), mean) <= TOL["bf16"]
+    assert _err(lse.double().numpy(), lse_ref) <= LSE_TOL
+
+
+def test_causal_row0_is_v0():
+    q, k, v = make_qkv(2, 4, 500, 500, 128, "bf16", seed=23)
+    o, lse = _run(q, k, v, True, 1.0 / math.sqrt(128))
+    assert torch.equal(o[:, :, 0], v[:, :, 0])
+    s00 = (q[:, :, 0].double() * k[:, :, 0].double()).sum(-1) / math.sqrt(128)
+    assert _err(lse[:, :, 0].double().numpy(), s00.numpy()) <= LSE_TOL
+
+
+def test_single_key():
+    q, k, v = make_qkv(1, 3, 200, 1, 64, "fp16", seed=24)
+    o, _ = _run(q, k, v, False, 0.125)
+    assert torch.equal(o, v.expand_as(o))
+
+
+def test_dominant_key():
+    q, k, v = make_qkv(1, 1, 256, 256, 64, "fp16", seed=25)
+    i, j = 77, 200
+    qi = q[0, 0, i].double()
+    k[0, 0, j] = (30.0 * qi / qi.norm()).half()  # gap of ~30 / sqrt(64) * |q_i| in the exponent
+    o, _ = _run(q, k, v, False, 1.0)
+    assert _err(o[0, 0, i].double().numpy(), v[0, 0, j].double().numpy()) <= TOL["fp16"]
+
+
+# ------------------------------------------------------------ memory safety, determinism
+
+@pytest.mark.parametrize("Nq,d,dtype", [(400, 64, "fp16"), (129, 128, "bf16"), (1, 64, "bf16")])
+def test_canary_bands(Nq, d, dtype):
+    """Rows past Nq, and memory around O and lse, are never written."""
+    B, H = 2, 3
+    q, k, v = make_qkv(B, H, Nq, 300, d, dtype, seed=26)
+    t = q.dtype
+    pad = 4096
+    n_o = B * H * Nq * d
+    o_buf = torch.full((n_o + 2 * pad,), 0, dtype=torch.int16, device="cuda")
+    o_buf.fill_(SENTINEL)
+    o_buf = o_buf.view(t)
+    l_buf = torch.full((B * H * Nq + 2 * pad,), float("nan"), dtype=torch.float32, device="cuda")
+    o = o_buf[pad:pad + n_o].view(B, H, Nq, d)
+    lse = l_buf[pad:pad + B * H * Nq].view(B, H, Nq)
+    A.forward(q.cuda(), k.cuda(), v.cuda(), causal=True, out=o, lse=lse)
+    torch.cuda.synchronize()
+    ob = o_buf.view(torch.int16).cpu()
+    assert (ob[:pad] == SENTINEL).all() and (ob[pad + n_o:] == SENTINEL).all()
+    lb = l_buf.cpu()
+    assert torch.isnan(lb[:pad]).all() and torch.isnan(lb[pad + B * H * Nq:]).all()
+    assert torch.isfinite(o.float()).all() and torch.isfinite(lse).all()
+    o_ref, l_ref = oracle.attention_f64(q, k, v, 1.0 / math.sqrt(d), True)
+    assert _err(o.cpu().double().numpy(), o_ref) <= TOL[dtype]
+    assert _err(lse.cpu().double().numpy(), l_ref) <= LSE_TOL
+
+
+def test_lse_null_skips_lse():
+    q, k, v = make_qkv(1, 2, 200, 200, 64, "fp16", seed=27)
+    o, lse = A.forward(q.cuda(), k.cuda(), v.cuda(), causal=False, return_lse=False)
+    assert lse is None
+    o2, _ = A.forward(q.cuda(), k.cuda(), v.cuda(), causal=False)
+    assert torch.equal(o, o2)
+
+
+@pytest.mark.parametrize("idx", [1, 3])
+def test_deterministic(idx):
+    w = WORKLOADS[idx]
+    q, k, v = (t.cuda() for t in make_workload_qkv(w))
+    o1, l1 = A.forward(q, k, v, causal=w.causal)
+    o2, l2 = A.forward(q, k, v, causal=w.causal)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_host_entry_matches_device_entry():
+    w = WORKLOADS[0]
+    q, k, v = make_workload_qkv(w)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32).pin_memory()
+    qd, kd, vd = (torch.empty_like(t, device="cuda") for t in (q, k, v))
+    od = torch.empty_like(qd)
+    ld = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device="cuda")
+    A.forward_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, causal=w.causal)
+    torch.cuda.synchronize()
+    o, lse = A.forward(q.cuda(), k.cuda(), v.cuda(), causal=w.causal)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, o.cpu()) and torch.equal(lh, lse.cpu())
+
+
+def test_device_errors_do_not_launch():
+    q = torch.zeros(1, 1, 8, 64, dtype=torch.float16, device="cuda")
+    base = q.data_ptr()
+    st = A.attn_fwd(base + 2, base, base, base, None, 1, 1, 8, 8, 64, 0.1, 0, 0, 0)
+    assert st == 5
+    st = A.attn_fwd(base, base, base, base, None, 1, 1, 8, 8, 80, 0.1, 0, 0, 0)
+    assert st == 3
+    assert A.attn_get_device_status()[0] == 0
