@@ -1,0 +1,428 @@
+#!/usr/bin/env python3
+"""Benchmark of the sm_100a exact attention forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload NAME] [--no-per-workload]
+
+One step = one attention forward (the whole hot path) over one batch of the
+workload: by default the 40x40 YOLO neck attention, B=16, H=4, Nq=Nk=1600,
+d=64, fp16, non-causal.  Inputs are seeded synthetic N(0,1) tensors resident
+in HBM; L2 (126 MB) is flushed by a 256 MiB write before every timed step
+because these inputs are smaller than L2.  Each step is timed with CUDA
+events on the launching stream; the timed region is bracketed by a barrier
+and a device synchronisation, and multi-GPU runs report the max over ranks.
+With N > 1 (torchrun), every rank runs its own copy of the workload over
+its own (batch, head) slice -- the method has no exchange step, so there is
+no collective on the data path (weak scaling).
+
+Rank 0 prints one JSON line.  ``--impl reference`` times the float64 CPU
+oracle instead (the slow baseline), on a bounded sample of the workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOPS & % of B200 roofline; µs/call at YOLO shapes"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+DEFAULT_WORKLOAD = "yolo_neck_40x40_b16"
+FLUSH_BYTES = 256 << 20
+KERNEL_SOURCES = ["exact_attention_153_b200/csrc/attn_fwd_sm100.cuh",
+                  "exact_attention_153_b200/csrc/sm100_ptx.cuh",
+                  "exact_attention_153_b200/csrc/attn_api.cu"]
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "attn_fwd_kernel_traffic.json")
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        p["source"] = "measured"
+        return p
+    p = dict(FALLBACK_PEAKS)
+    p["source"] = "fallback"
+    return p
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if still current."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        doc = json.load(f)
+    ent = doc.get("workloads", {}).get(workload)
+    if not ent or ent.get("kernel_source_sha") != kernel_source_sha():
+        return None
+    return ent.get("dram_bytes_per_launch")
+
+
+def roofline(w, t_s, peaks, sustained=False):
+    """Which roof bounds this workload and how close one launch gets to it."""
+    flops_peak = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"] * 1e12
+    bw_peak = peaks["hbm_gbs"] * 1e9
+    if w.flops / w.bytes >= flops_peak / bw_peak:
+        achieved = w.flops / t_s / 1e12
+        peak = flops_peak / 1e12
+        return {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4)}
+    achieved = w.bytes / t_s / 1e9
+    peak = bw_peak / 1e9
+    return {"bound": "hbm", "achieved": round(achieved, 1), "peak": round(peak, 1),
+            "unit": "GB/s", "frac": round(achieved / peak, 4)}
+
+
+class ClockSampler(threading.Thread):
+    """Polls SM clock and clock-event reasons through NVML during the timed region."""
+
+    REASONS = {
+        0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+        0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+        0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown",
+        0x100: "display_clock_setting",
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        super().__init__(daemon=True)
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._halt = threading.Event()
+        self.error = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # NVML missing: report it, keep benchmarking
+            self.nv = None
+            self.error = repr(e)
+
+    def run(self):
+        if self.nv is None:
+            return
+        nv = self.nv
+        while not self._halt.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                self.reasons |= nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            except Exception as e:
+                self.error = repr(e)
+                return
+            time.sleep(self.period)
+
+    def stop(self):
+        self._halt.set()
+        self.join(timeout=2)
+
+    def summary(self):
+        reasons = [name for bit, name in self.REASONS.items() if self.reasons & bit]
+        out = {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+               "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples),
+               "source": "nvml"}
+        if self.error:
+            out["error"] = self.error
+        return out
+
+
+def cpu_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def time_oracle_sample(w, q, k, v, budget_s=12.0, max_heads=None):
+    """Run the float64 oracle over whole (batch, head) slices until the budget is spent."""
+    import numpy as np
+    import oracle
+    rows = np.arange(w.Nq)
+    heads = [(b, h) for b in range(w.B) for h in range(w.H)]
+    if max_heads is not None:
+        heads = heads[:max_heads]
+    done = 0
+    t0 = time.perf_counter()
+    for b, h in heads:
+        oracle.attention_head_rows(q[b, h], k[b, h], v[b, h], w.scale, w.causal, rows)
+        done += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    flops = w.flops * done / len(heads) if max_heads is None else w.flops * done / (w.B * w.H)
+    return flops, dt, done
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else None
+    except Exception:
+        return None
+
+
+def run_reference(args, w):
+    """The oracle as it stands, on the host cores: each step one bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from seeded_inputs import make_workload_qkv
+    q, k, v = make_workload_qkv(w)
+    heads_per_step = max(1, min(w.B * w.H, 8))
+    for _ in range(args.warmup):
+        time_oracle_sample(w, q, k, v, budget_s=1e9, max_heads=heads_per_step)
+    tot_flops = tot_t = 0.0
+    for _ in range(args.steps):
+        f, dt, _ = time_oracle_sample(w, q, k, v, budget_s=1e9, max_heads=heads_per_step)
+        tot_flops += f
+        tot_t += dt
+    value = tot_flops / tot_t / 1e12
+    cores = blas_threads() or cpu_cores()
+    sample = (f"{heads_per_step} of {w.B * w.H} (batch, head) slices per step, all "
+              f"{w.Nq} query rows each, float64 numpy")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", args.gpus)), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1))",
+        "config": dict(w.as_config(), parallelism="host cores, rank 0 only"),
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the context timings of the other workloads")
+    ap.add_argument("--cpu-budget", type=float, default=12.0,
+                    help="seconds of float64 oracle work for cpu_baseline")
+    ap.add_argument("--kernel-only", action="store_true",
+                    help="time only the device loop (no e2e, CPU baseline or context timings);"
+                         " used for ncu captures")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    from seeded_inputs import workload
+    w = workload(args.workload)
+    if args.impl == "reference":
+        return run_reference(args, w)
+
+    import torch
+    import torch.distributed as dist
+    import exact_attention_153_b200 as attn
+    from seeded_inputs import Workload, make_qkv
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120))
+    dev = torch.device("cuda", torch.cuda.current_device())
+    stream = torch.cuda.current_stream()
+    peaks = load_peaks()
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # each rank: its own seeded copy of the workload (weak scaling over (batch, head))
+    q, k, v = make_qkv(w.B, w.H, w.Nq, w.Nk, w.d, w.dtype, w.seed + 1000 * rank, w.qk_scale)
+    qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
+    od = torch.empty_like(qd)
+    ld = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    code = attn.ATTN_BF16 if w.dtype == "bf16" else attn.ATTN_FP16
+    sh = stream.cuda_stream
+
+    def step():
+        st = attn.attn_fwd(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
+                           ld.data_ptr(), w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, code, sh)
+        if st != 0:
+            raise attn.AttnError(st)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    for e0, e1 in evs:
+        flush.zero_()
+        e0.record(stream)
+        step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    sampler.stop()
+    kernel_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    total_ms = sum(kernel_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    st, word = attn.attn_get_device_status(sh)
+    if st != 0:
+        raise attn.AttnError(st, f"device status {word:#x}")
+    if args.kernel_only:
+        if rank == 0:
+            ms = total_ms / args.steps
+            print(json.dumps({"workload": w.name, "us_per_call": round(ms * 1e3, 2),
+                              "tflops": round(world * w.flops / (ms * 1e-3) / 1e12, 2),
+                              "n_gpus": world, "steps": args.steps}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
+
+    # ---------------------------------------------------------------- end to end
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32).pin_memory()
+
+    def e2e_step():
+        st = attn.attn_fwd_host(qh.data_ptr(), kh.data_ptr(), vh.data_ptr(), oh.data_ptr(),
+                                lh.data_ptr(), qd.data_ptr(), kd.data_ptr(), vd.data_ptr(),
+                                od.data_ptr(), ld.data_ptr(), w.B, w.H, w.Nq, w.Nk, w.d, w.scale,
+                                w.causal, code, sh)
+        if st != 0:
+            raise attn.AttnError(st, "attn_fwd_host")
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e_start.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    e_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    e2e_ms = e_start.elapsed_time(e_end)
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    ms_per_step = total_ms / args.steps
+    value = world * w.flops * args.steps / (total_ms * 1e-3) / 1e12
+    e2e_value = world * w.flops * args.steps / (e2e_ms * 1e-3) / 1e12
+    per_launch_s = ms_per_step * 1e-3
+    roof = roofline(w, per_launch_s, peaks)
+    roof["peak_source"] = peaks["source"]
+    roof["traffic"] = recorded_traffic(w.name)
+    roof["algorithmic_flops_per_launch"] = w.flops
+    roof["algorithmic_bytes_per_launch"] = w.bytes
+
+    per_workload = None
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_per_workload:
+        per_workload = context_timings(attn, torch, dev, peaks)
+    if rank == 0:
+        flops, dt, done = time_oracle_sample(w, q, k, v, budget_s=args.cpu_budget)
+        cpu = {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": blas_threads() or cpu_cores(),
+               "kind": "oracle",
+               "sample": f"{done} of {w.B * w.H} (batch, head) slices of {w.name}, all "
+                         f"{w.Nq} rows each, float64 numpy, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 3), "unit": "TFLOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+            "us_per_call": round(ms_per_step * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic (seeded N(0,1), recipe in seeded_inputs)",
+            "config": dict(w.as_config(), l2="flushed before every timed step (256 MiB write)",
+                           parallelism=f"dp{world} over (batch, head) slices, no collective"),
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS",
+                    "h2d_bytes_per_step": int(q.numel() + k.numel() + v.numel()) * 2,
+                    "d2h_bytes_per_step": int(q.numel()) * 2 + w.B * w.H * w.Nq * 4,
+                    "ms_per_step": round(e2e_ms / args.steps, 4),
+                    "path": "attn_fwd_host: pinned host -> device, kernel, device -> host"},
+            "gpu_launches": args.steps,
+            "clocks": sampler.summary(),
+            "kernel_source_sha": kernel_source_sha(),
+        }
+        if per_workload is not None:
+            line["per_workload"] = per_workload
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+def context_timings(attn, torch, dev, peaks, steps=10):
+    """µs/call, TFLOPS and roofline fraction of every workload (L2 flushed each call)."""
+    from seeded_inputs import WORKLOADS, make_workload_qkv
+    out = {}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for w in WORKLOADS:
+        q, k, v = (t.to(dev) for t in make_workload_qkv(w))
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+        for _ in range(3):
+            attn.forward(q, k, v, causal=w.causal, out=o, lse=lse)
+        times = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            attn.forward(q, k, v, causal=w.causal, out=o, lse=lse)
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1))
+        us = statistics.median(times) * 1e3
+        r = roofline(w, us * 1e-6, peaks)
+        out[w.name] = {"us_per_call": round(us, 2), "tflops": round(w.flops / (us * 1e-6) / 1e12, 2),
+                       "bound": r["bound"], "frac": r["frac"],
+                       "frac_of_sustained": roofline(w, us * 1e-6, peaks, sustained=True)["frac"]}
+        del q, k, v, o, lse
+    return out
+
+
+if __name__ == "__main__":
+    sys.exit(main())

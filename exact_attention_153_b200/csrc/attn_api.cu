@@ -85,11 +85,13 @@ void fill_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, att
   const int q_tiles = ceil_div(Nq, BLOCK_M);
   const int q_pairs = ceil_div(q_tiles, 2);
   const int kv_tiles = ceil_div(Nk, BLOCK_N);
-  const long long units = static_cast<long long>(B) * H * q_pairs;
+  const int units_per_head = causal ? (q_pairs + 1) / 2 : q_pairs;
+  const long long units = static_cast<long long>(B) * H * units_per_head;
   out->num_q_tiles = q_tiles;
   out->num_q_pairs = q_pairs;
   out->num_kv_tiles = kv_tiles;
   out->num_units = static_cast<int>(units);
+  out->units_per_head = units_per_head;
   out->grid = static_cast<int>(units < num_sms ? units : num_sms);
   out->block = NUM_THREADS;
   out->smem_bytes = d == 64 ? SmemLayout<64>::BYTES : SmemLayout<128>::BYTES;
@@ -225,6 +227,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   prm.BH = static_cast<int>(BH);
   prm.num_q_pairs = plan.num_q_pairs;
   prm.num_kv_tiles = plan.num_kv_tiles;
+  prm.units_per_head = plan.units_per_head;
   prm.num_units = plan.num_units;
   prm.causal = causal ? 1 : 0;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);

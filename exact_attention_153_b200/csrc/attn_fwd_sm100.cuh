@@ -44,10 +44,21 @@ namespace attn_sm100 {
 
 constexpr int BLOCK_M = 128;     // query rows per Q tile (= TMEM lanes)
 constexpr int BLOCK_N = 128;     // keys per K / V tile
-constexpr int NUM_THREADS = 320; // 8 softmax warps + MMA warp + load warp
+// 12 warps = 3 warpgroups: two softmax warpgroups (warps 0-3, 4-7) and one
+// producer warpgroup (warp 8 issues MMAs, warp 9 issues TMA loads, warps 10-11
+// idle).  Launched at 168 registers per thread (the per-SM-sub-partition
+// limit for 3 warps each); the producer warpgroup then gives registers up
+// and the softmax warpgroups take them: 2 * 128 * 200 + 128 * 96 = 63488 <=
+// 384 * 168, so the increase never waits on registers that do not exist.
+constexpr int NUM_THREADS = 384;
 constexpr int MMA_WARP = 8;
 constexpr int LOAD_WARP = 9;
+constexpr uint32_t SOFTMAX_REGS = 200;
+constexpr uint32_t PRODUCER_REGS = 96;
+static_assert(2 * 128 * SOFTMAX_REGS + 128 * PRODUCER_REGS <= NUM_THREADS * 168,
+              "register split exceeds the launch budget");
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
+constexpr float RESCALE_LOG2 = 8.0f;  // lazy-rescale threshold for the running max
 
 // Device status word: 0 = healthy; otherwise 0x80000000 | site.
 __device__ unsigned int g_attn_status = 0;
@@ -69,7 +80,8 @@ struct FwdParams {
   int Nq, Nk, BH;
   int num_q_pairs;  // ceil(ceil(Nq / 128) / 2)
   int num_kv_tiles; // ceil(Nk / 128)
-  int num_units;    // BH * num_q_pairs
+  int units_per_head; // causal: ceil(num_q_pairs / 2); else num_q_pairs
+  int num_units;    // BH * units_per_head
   int causal;
   float scale_log2; // scale * log2(e)
 };
@@ -108,19 +120,30 @@ struct Unit {
   int nmax;
 };
 
-// Work-unit order.  Causal: heaviest Q pairs first (longest-processing-time
-// order) so the persistent CTAs finish together.  Non-causal: the Q pairs of
-// one head are adjacent, so CTAs running at the same time share that head's
-// K/V through L2.
-__device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
+// Work schedule.  A work unit belongs to one (batch, head) and holds one or
+// two "items"; an item is a pair of adjacent 128-row Q tiles.  CTA c takes
+// units c, c + grid, c + 2 grid, ...; consecutive units belong to the same
+// head, so CTAs running at the same time share that head's K/V through L2.
+//   non-causal: one item per unit, every item costs the same.
+//   causal: unit b of a head holds Q pair (n_pairs - 1 - b) and its mirror b,
+//     heaviest first; the two together always visit about n_pairs + 1 K/V
+//     tiles, so every unit costs the same and the persistent CTAs finish
+//     together.
+__device__ __forceinline__ int unit_items(const FwdParams& p, int u) {
+  if (!p.causal) return 1;
+  const int b = u % p.units_per_head;
+  return (b != p.num_q_pairs - 1 - b) ? 2 : 1;
+}
+
+__device__ __forceinline__ Unit decode_item(const FwdParams& p, int u, int item) {
   Unit w;
   int qp;
+  w.bh = u / p.units_per_head;
+  const int b = u % p.units_per_head;
   if (p.causal) {
-    qp = p.num_q_pairs - 1 - u / p.BH;
-    w.bh = u % p.BH;
+    qp = item == 0 ? p.num_q_pairs - 1 - b : b;
   } else {
-    w.bh = u / p.num_q_pairs;
-    qp = u % p.num_q_pairs;
+    qp = b;
   }
   w.q0 = qp * 2 * BLOCK_M;
 #pragma unroll
@@ -141,29 +164,28 @@ __device__ __forceinline__ Unit decode_unit(const FwdParams& p, int u) {
   return w;
 }
 
-// Bounded wait on one mbarrier phase.  Returns false on timeout (status word
-// set, abort flag raised) or, when honour_abort, once another role aborted.
-__device__ __noinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                        uint32_t site, bool honour_abort) {
-  const uint64_t t0 = global_timer_ns();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 128; ++i) {
-      if (mbar_try_wait(bar, parity)) return true;
-    }
-    if (honour_abort && *abort_flag) return false;
-    if (global_timer_ns() - t0 > WAIT_LIMIT_NS) {
-      atomicCAS(&g_attn_status, 0u, 0x80000000u | site);
-      *abort_flag = 1;
-      return false;
+// Bounded wait on one mbarrier phase, fully inlined (a call here would make
+// the compiler save live registers to local memory on every slow wait).
+// Returns false on timeout (status word set, abort flag raised) or, when
+// honour_abort, once another role has aborted.
+__device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                           uint32_t site, bool honour_abort = true) {
+  uint32_t spins = 0;
+  uint64_t t0 = 0;
+  while (!mbar_try_wait(bar, parity)) {
+    if ((++spins & 1023u) == 0) {
+      const uint64_t now = global_timer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > WAIT_LIMIT_NS) {
+        atomicCAS(&g_attn_status, 0u, 0x80000000u | site);
+        *abort_flag = 1;
+        return false;
+      }
+      if (honour_abort && *abort_flag) return false;
     }
   }
-}
-
-__device__ __forceinline__ bool wait_fast(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          uint32_t site) {
-  if (mbar_try_wait(bar, parity)) return true;
-  return wait_phase(bar, parity, abort_flag, site, true);
+  return true;
 }
 
 template <int D, bool BF16>
@@ -211,38 +233,63 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp == LOAD_WARP) {
-    // ------------------------------------------------------------- TMA producer
-    if (lane == 0) {
-      const uint32_t q_smem = sbase + L::Q_OFF;
-      const uint32_t kv_smem = sbase + L::KV_OFF;
+  if (warp >= 8) {
+    regs_decrease<PRODUCER_REGS>();
+    // The producer warps run their loops on all 32 lanes, so every address,
+    // coordinate and descriptor is warp-uniform and stays in uniform
+    // registers; one elected lane issues the TMA and tcgen05 instructions
+    // (a loop on one lane would have to move each operand into uniform
+    // registers before every MMA, which made the issue the bottleneck).
+    const bool leader = elect_one();
+    const uint32_t q_smem = sbase + L::Q_OFF;
+    const uint32_t kv_smem = sbase + L::KV_OFF;
+    auto warp_wait = [&](uint32_t b, uint32_t parity, uint32_t site) -> bool {
+      const bool r = wait_phase(b, parity, abort_flag, site);
+      return __all_sync(0xffffffffu, r);
+    };
+    if (warp == LOAD_WARP) {
+      // ----------------------------------------------------------- TMA producer
       uint32_t kv_it = 0, units = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-        const Unit w = decode_unit(p, u);
-        if (units > 0) {
-          ok = wait_fast(bar(L::Q_EMPTY), (units - 1) & 1, abort_flag, SITE_LOAD_Q_EMPTY);
-          if (!ok) break;
-        }
-        mbar_arrive_expect_tx(bar(L::Q_FULL), 2 * L::TILE_BYTES);
-        for (int t = 0; t < 2; ++t)
-          for (int h = 0; h < L::HALVES; ++h)
-            tma_load_3d(q_smem + t * L::TILE_BYTES + h * L::HALF_BYTES, &tm_q, bar(L::Q_FULL),
-                        h * 64, w.q0 + t * BLOCK_M, w.bh);
-        ++units;
-        for (int j = 0; ok && j < w.nmax; ++j) {
-          for (int which = 0; which < 2; ++which) {
-            const uint32_t st = kv_it % L::STAGES;
-            const uint32_t ph = (kv_it / L::STAGES) & 1;
-            if (kv_it >= static_cast<uint32_t>(L::STAGES)) {
-              ok = wait_fast(bar(L::KV_EMPTY + st), ph ^ 1, abort_flag, SITE_LOAD_KV_EMPTY);
-              if (!ok) break;
+        const int items = unit_items(p, u);
+        for (int item = 0; ok && item < items; ++item) {
+          const Unit w = decode_item(p, u, item);
+          if (units > 0) {
+            ok = warp_wait(bar(L::Q_EMPTY), (units - 1) & 1, SITE_LOAD_Q_EMPTY);
+            if (!ok) break;
+          }
+          if (leader) {
+            mbar_arrive_expect_tx(bar(L::Q_FULL), 2 * L::TILE_BYTES);
+#pragma unroll
+            for (int t = 0; t < 2; ++t)
+#pragma unroll
+              for (int h = 0; h < L::HALVES; ++h)
+                tma_load_3d(q_smem + t * L::TILE_BYTES + h * L::HALF_BYTES, &tm_q, bar(L::Q_FULL),
+                            h * 64, w.q0 + t * BLOCK_M, w.bh);
+          }
+          __syncwarp();
+          ++units;
+          for (int j = 0; ok && j < w.nmax; ++j) {
+#pragma unroll
+            for (int which = 0; which < 2; ++which) {
+              const uint32_t st = kv_it % L::STAGES;
+              const uint32_t ph = (kv_it / L::STAGES) & 1;
+              if (kv_it >= static_cast<uint32_t>(L::STAGES)) {
+                ok = warp_wait(bar(L::KV_EMPTY + st), ph ^ 1, SITE_LOAD_KV_EMPTY);
+                if (!ok) break;
+              }
+              if (leader) {
+                mbar_arrive_expect_tx(bar(L::KV_FULL + st), L::TILE_BYTES);
+#pragma unroll
+                for (int h = 0; h < L::HALVES; ++h)
+                  tma_load_3d(kv_smem + st * L::TILE_BYTES + h * L::HALF_BYTES,
+                              which ? &tm_v : &tm_k, bar(L::KV_FULL + st), h * 64, j * BLOCK_N,
+                              w.bh);
+              }
+              __syncwarp();
+              ++kv_it;
             }
-            mbar_arrive_expect_tx(bar(L::KV_FULL + st), L::TILE_BYTES);
-            for (int h = 0; h < L::HALVES; ++h)
-              tma_load_3d(kv_smem + st * L::TILE_BYTES + h * L::HALF_BYTES, which ? &tm_v : &tm_k,
-                          bar(L::KV_FULL + st), h * 64, j * BLOCK_N, w.bh);
-            ++kv_it;
           }
         }
       }
@@ -252,119 +299,135 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         wait_phase(bar(L::KV_FULL + i % L::STAGES), (i / L::STAGES) & 1, abort_flag, SITE_DRAIN,
                    false);
       if (units > 0) wait_phase(bar(L::Q_FULL), (units - 1) & 1, abort_flag, SITE_DRAIN, false);
-    }
-    __syncwarp();
-  } else if (warp == MMA_WARP) {
-    // ------------------------------------------------------------- MMA issuer
-    if (lane == 0) {
+      __syncwarp();
+    } else if (warp == MMA_WARP) {
+      // ----------------------------------------------------------- MMA issuer
       constexpr uint32_t IDESC_S = idesc_f16(BF16, false, false, BLOCK_M, BLOCK_N);
       constexpr uint32_t IDESC_O = idesc_f16(BF16, false, true, BLOCK_M, D);
-      const uint32_t q_smem = sbase + L::Q_OFF;
-      const uint32_t kv_smem = sbase + L::KV_OFF;
-
       // S_t = Q_t K^T: both operands K-major (head dim contiguous), 128-byte
       // swizzle, 8-row groups 1024 bytes apart; each k-step covers 16
       // elements = 32 bytes of a 128-byte row, the head dim > 64 continues in
-      // the next 16 KB slab.
-      auto issue_s = [&](int t, uint32_t stage) {
-        const uint32_t qa = q_smem + t * L::TILE_BYTES;
-        const uint32_t ka = kv_smem + stage * L::TILE_BYTES;
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk / 4) * L::HALF_BYTES + (kk % 4) * 32;
-          mma_ss(tmem_base + L::S_COL + 128 * t, sw128_desc(qa + off, 16, 1024),
-                 sw128_desc(ka + off, 16, 1024), IDESC_S, kk > 0 ? 1u : 0u);
-        }
-      };
+      // the next 16 KB slab.  Descriptors are built once; a k-step or a ring
+      // slot only adds (byte offset >> 4) to the start-address field (every
+      // address stays below 256 KB, so the add never carries out of it).
+      const uint64_t q_desc = sw128_desc(q_smem, 16, 1024);
+      const uint64_t k_desc = sw128_desc(kv_smem, 16, 1024);
       // O_t += P_t V: P from TMEM (16 keys = 8 columns per k-step), V
       // MN-major (head dim contiguous): 8-key groups 1024 bytes apart,
       // 64-column slabs 16 KB apart; each k-step advances 16 keys = 2 KB.
-      auto issue_pv = [&](int t, uint32_t stage, bool accumulate) {
-        const uint32_t va = kv_smem + stage * L::TILE_BYTES;
+      const uint64_t v_desc = sw128_desc(kv_smem, L::HALF_BYTES, 1024);
+      const uint32_t tmem_s = tmem_base + L::S_COL;
+      const uint32_t tmem_o = tmem_base + L::O_COL;
+
+      auto issue_s = [&](int t, uint32_t stage) {
+        const uint64_t a = q_desc + static_cast<uint32_t>(t * (L::TILE_BYTES >> 4));
+        const uint64_t b = k_desc + stage * static_cast<uint32_t>(L::TILE_BYTES >> 4);
+        if (leader) {
 #pragma unroll
-        for (int kk = 0; kk < BLOCK_N / 16; ++kk) {
-          mma_ts(tmem_base + L::O_COL + D * t, tmem_base + L::S_COL + 128 * t + kk * 8,
-                 sw128_desc(va + kk * 2048, L::HALF_BYTES, 1024), IDESC_O,
-                 (accumulate || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = ((kk / 4) * L::HALF_BYTES + (kk % 4) * 32) >> 4;
+            mma_ss(tmem_s + 128 * t, a + off, b + off, IDESC_S, kk > 0 ? 1u : 0u);
+          }
         }
+      };
+      auto issue_pv = [&](int t, uint32_t stage, bool accumulate) {
+        const uint64_t b = v_desc + stage * static_cast<uint32_t>(L::TILE_BYTES >> 4);
+        if (leader) {
+#pragma unroll
+          for (int kk = 0; kk < BLOCK_N / 16; ++kk)
+            mma_ts(tmem_o + D * t, tmem_s + 128 * t + kk * 8, b + kk * (2048 >> 4), IDESC_O,
+                   (accumulate || kk > 0) ? 1u : 0u);
+        }
+      };
+      auto commit = [&](uint32_t b) {
+        if (leader) mma_commit(b);
       };
 
       uint32_t kv_it = 0, q_phase = 0;
       uint32_t p_phase[2] = {0, 0};
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-        const Unit w = decode_unit(p, u);
-        ok = wait_fast(bar(L::Q_FULL), q_phase, abort_flag, SITE_MMA_Q_FULL);
-        if (!ok) break;
-        q_phase ^= 1;
-        {
-          const uint32_t st = kv_it % L::STAGES, ph = (kv_it / L::STAGES) & 1;
-          ++kv_it;
-          ok = wait_fast(bar(L::KV_FULL + st), ph, abort_flag, SITE_MMA_KV_FULL);
+        const int items = unit_items(p, u);
+        for (int item = 0; ok && item < items; ++item) {
+          const Unit w = decode_item(p, u, item);
+          ok = warp_wait(bar(L::Q_FULL), q_phase, SITE_MMA_Q_FULL);
           if (!ok) break;
-          tc_fence_after();
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (w.n[t] > 0) {
-              issue_s(t, st);
-              mma_commit(bar(L::S_FULL + t));
-            }
-          }
-          mma_commit(bar(L::KV_EMPTY + st));
-        }
-        for (int j = 0; ok && j < w.nmax; ++j) {
-          const uint32_t vst = kv_it % L::STAGES, vph = (kv_it / L::STAGES) & 1;
-          ++kv_it;
-          const bool has_next = j + 1 < w.nmax;
-          uint32_t kst = 0, kph = 0;
-          if (has_next) {
-            kst = kv_it % L::STAGES;
-            kph = (kv_it / L::STAGES) & 1;
+          q_phase ^= 1;
+          {
+            const uint32_t st = kv_it % L::STAGES, ph = (kv_it / L::STAGES) & 1;
             ++kv_it;
-          }
-          ok = wait_fast(bar(L::KV_FULL + vst), vph, abort_flag, SITE_MMA_KV_FULL);
-          if (!ok) break;
-          bool k_ready = false;
-#pragma unroll
-          for (int t = 0; t < 2; ++t) {
-            if (!ok || j >= w.n[t]) continue;
-            ok = wait_fast(bar(L::P_FULL + t), p_phase[t], abort_flag, SITE_MMA_P_FULL);
-            if (!ok) continue;
-            p_phase[t] ^= 1;
+            ok = warp_wait(bar(L::KV_FULL + st), ph, SITE_MMA_KV_FULL);
+            if (!ok) break;
             tc_fence_after();
-            issue_pv(t, vst, j > 0);
-            if (j + 1 < w.n[t]) {
-              if (!k_ready) {
-                ok = wait_fast(bar(L::KV_FULL + kst), kph, abort_flag, SITE_MMA_KV_FULL);
-                if (!ok) continue;
-                tc_fence_after();
-                k_ready = true;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (w.n[t] > 0) {
+                issue_s(t, st);
+                commit(bar(L::S_FULL + t));
               }
-              issue_s(t, kst);
-              mma_commit(bar(L::S_FULL + t));
-            } else {
-              mma_commit(bar(L::O_FULL + t));
             }
+            commit(bar(L::KV_EMPTY + st));
+            __syncwarp();
+          }
+          for (int j = 0; ok && j < w.nmax; ++j) {
+            const uint32_t vst = kv_it % L::STAGES, vph = (kv_it / L::STAGES) & 1;
+            ++kv_it;
+            const bool has_next = j + 1 < w.nmax;
+            uint32_t kst = 0, kph = 0;
+            if (has_next) {
+              kst = kv_it % L::STAGES;
+              kph = (kv_it / L::STAGES) & 1;
+              ++kv_it;
+            }
+            ok = warp_wait(bar(L::KV_FULL + vst), vph, SITE_MMA_KV_FULL);
+            if (!ok) break;
+            bool k_ready = false;
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+              if (!ok || j >= w.n[t]) continue;
+              ok = warp_wait(bar(L::P_FULL + t), p_phase[t], SITE_MMA_P_FULL);
+              if (!ok) continue;
+              p_phase[t] ^= 1;
+              tc_fence_after();
+              issue_pv(t, vst, j > 0);
+              if (j + 1 < w.n[t]) {
+                if (!k_ready) {
+                  ok = warp_wait(bar(L::KV_FULL + kst), kph, SITE_MMA_KV_FULL);
+                  if (!ok) continue;
+                  tc_fence_after();
+                  k_ready = true;
+                }
+                issue_s(t, kst);
+                commit(bar(L::S_FULL + t));
+              } else {
+                commit(bar(L::O_FULL + t));
+              }
+              __syncwarp();
+            }
+            if (!ok) break;
+            commit(bar(L::KV_EMPTY + vst));
+            if (has_next) {
+              if (!k_ready) {
+                ok = warp_wait(bar(L::KV_FULL + kst), kph, SITE_MMA_KV_FULL);
+                if (!ok) break;
+              }
+              commit(bar(L::KV_EMPTY + kst));
+            }
+            __syncwarp();
           }
           if (!ok) break;
-          mma_commit(bar(L::KV_EMPTY + vst));
-          if (has_next) {
-            if (!k_ready) {
-              ok = wait_fast(bar(L::KV_FULL + kst), kph, abort_flag, SITE_MMA_KV_FULL);
-              if (!ok) break;
-            }
-            mma_commit(bar(L::KV_EMPTY + kst));
-          }
+          commit(bar(L::Q_EMPTY));
+          __syncwarp();
         }
-        if (!ok) break;
-        mma_commit(bar(L::Q_EMPTY));
       }
       // All MMAs (and their commits) must be finished before TMEM is freed.
-      mma_commit(bar(L::DRAIN));
+      commit(bar(L::DRAIN));
+      __syncwarp();
       wait_phase(bar(L::DRAIN), 0, abort_flag, SITE_DRAIN, false);
+      __syncwarp();
     }
-    __syncwarp();
   } else {
+    regs_increase<SOFTMAX_REGS>();
     // ------------------------------------------------------------- softmax
     const int t = warp / 4;
     const int quarter = warp % 4;
@@ -376,7 +439,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t s_phase = 0, o_phase = 0;
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-      const Unit w = decode_unit(p, u);
+     const int items = unit_items(p, u);
+     for (int item = 0; ok && item < items; ++item) {
+      const Unit w = decode_item(p, u, item);
       const int n = t ? w.n[1] : w.n[0];
       if (n == 0) continue;
       const int q_start = w.q0 + t * BLOCK_M;
@@ -385,7 +450,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int last_key = p.causal ? min(p.Nk - 1, row) : (p.Nk - 1);
       float m = -INFINITY, l = 0.f;
       for (int j = 0; j < n; ++j) {
-        ok = wait_fast(bar(L::S_FULL + t), s_phase, abort_flag, SITE_SOFTMAX_S_FULL);
+        ok = wait_phase(bar(L::S_FULL + t), s_phase, abort_flag, SITE_SOFTMAX_S_FULL);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         s_phase ^= 1;
@@ -415,29 +480,38 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           mx3 = fmaxf(mx3, s[c + 3]);
         }
         const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
-        const float m_new = fmaxf(m, mx * sl2);
+        // The running max only moves when the tile raises it by more than
+        // RESCALE_LOG2 (base 2): until then exponents stay below
+        // 2^RESCALE_LOG2 and O, l and lse keep using the same stale max, so
+        // the result is unchanged while most O rescales are skipped.
+        const float m_cand = fmaxf(m, mx * sl2);
+        const bool raise = m_cand > m + RESCALE_LOG2;
+        const float m_new = raise ? m_cand : m;
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = ex2_approx(m - m_use);
+        const float alpha = raise ? ex2_approx(m - m_use) : 1.f;
         const float neg_m = -m_use;
 
+        // P = 2^(s * scale * log2 e - m), packed two keys per 32-bit TMEM
+        // column (even key in the low half), written over S in 16-column
+        // chunks so each chunk's S registers die as it is stored.
         float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
-        for (int hblk = 0; hblk < 2; ++hblk) {
-          uint32_t pk[32];
+        for (int chunk = 0; chunk < 4; ++chunk) {
+          uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            const float a = ex2_approx(fmaf(s[64 * hblk + 2 * c], sl2, neg_m));
-            const float b = ex2_approx(fmaf(s[64 * hblk + 2 * c + 1], sl2, neg_m));
+          for (int c = 0; c < 16; ++c) {
+            const float a = ex2_approx(fmaf(s[32 * chunk + 2 * c], sl2, neg_m));
+            const float b = ex2_approx(fmaf(s[32 * chunk + 2 * c + 1], sl2, neg_m));
             sum0 += a;
             sum1 += b;
             pk[c] = pack2<BF16>(a, b);
           }
-          tmem_st32(tS + 32 * hblk, pk);
+          tmem_st16(tS + 16 * chunk, pk);
         }
         l = l * alpha + (sum0 + sum1);
         m = m_new;
 
-        if (j > 0 && __any_sync(0xffffffffu, alpha < 1.f)) {
+        if (__any_sync(0xffffffffu, raise && j > 0)) {
 #pragma unroll
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o[32];
@@ -455,7 +529,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (!ok) break;
 
       // ----------------------------------------------------------- epilogue
-      ok = wait_fast(bar(L::O_FULL + t), o_phase, abort_flag, SITE_SOFTMAX_O_FULL);
+      ok = wait_phase(bar(L::O_FULL + t), o_phase, abort_flag, SITE_SOFTMAX_O_FULL);
       ok = __all_sync(0xffffffffu, ok);
       if (!ok) break;
       o_phase ^= 1;
@@ -482,6 +556,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       if (p.lse != nullptr && in_range)
         p.lse[static_cast<size_t>(w.bh) * p.Nq + row] = (m + lg2_approx(l)) * 0.69314718055994531f;
       tc_fence_before();
+     }
     }
   }
 

@@ -56,9 +56,11 @@ typedef enum {
 /* Launch geometry for one call (see attn_plan). */
 typedef struct {
   int num_q_tiles;   /* ceil(Nq / 128): 128-row query tiles per (batch, head)            */
-  int num_q_pairs;   /* ceil(num_q_tiles / 2): a work unit is two query tiles             */
+  int num_q_pairs;   /* ceil(num_q_tiles / 2): query tiles are processed in pairs         */
   int num_kv_tiles;  /* ceil(Nk / 128): 128-key tiles per (batch, head)                   */
-  int num_units;     /* B * H * num_q_pairs work units                                    */
+  int units_per_head; /* work units per (batch, head): num_q_pairs, or for causal
+                         ceil(num_q_pairs / 2) (a heavy query pair with its mirror)          */
+  int num_units;     /* B * H * units_per_head work units                                 */
   int grid;          /* persistent CTAs launched: min(num_units, SM count)                */
   int block;         /* threads per CTA                                                   */
   int smem_bytes;    /* dynamic shared memory per CTA                                     */

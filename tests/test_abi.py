@@ -120,16 +120,21 @@ def test_host_entry_argument_errors():
 def test_plan_geometry():
     p = A.attn_plan(1, 2, 400, 400, 64, 0, 148)
     assert (p["num_q_tiles"], p["num_q_pairs"], p["num_kv_tiles"], p["num_units"]) == (4, 2, 4, 4)
-    assert p["grid"] == 4 and p["block"] == 320
+    assert p["grid"] == 4 and p["block"] == 384
     assert p["qk_tile_products"] == 2 * 4 * 4
     p = A.attn_plan(16, 4, 1600, 1600, 64, 0, 148)
     assert (p["num_q_tiles"], p["num_q_pairs"], p["num_units"], p["grid"]) == (13, 7, 448, 148)
     assert p["smem_bytes"] <= 232448
     p = A.attn_plan(32, 16, 2048, 2048, 64, 1, 148)
+    # causal: a unit is a heavy query pair with its mirror (8 pairs -> 4 units per head)
+    assert (p["num_q_pairs"], p["units_per_head"], p["num_units"]) == (8, 4, 32 * 16 * 4)
     # causal: query tile i visits key tiles 0..i
     assert p["qk_tile_products"] == 32 * 16 * sum(range(1, 17))
     p = A.attn_plan(1, 32, 32768, 32768, 128, 1, 148)
     assert p["stages"] == 4 and p["smem_bytes"] <= 232448
+    assert (p["num_q_pairs"], p["units_per_head"]) == (128, 64)
+    p2 = A.attn_plan(1, 1, 3 * 256, 3 * 256, 64, 1, 148)  # odd pair count: middle pair alone
+    assert (p2["num_q_pairs"], p2["units_per_head"], p2["num_units"]) == (3, 2, 2)
     assert p["qk_tile_products"] == 32 * sum(range(1, 257))
     # ragged causal with Nq != Nk (top-left): rows past Nk see every key
     p = A.attn_plan(1, 1, 300, 200, 64, 1, 148)
