@@ -459,7 +459,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * c));
-        tmem_wait_ld();
+        tmem_wait_ld_regs(sr);
         float s[128];
 #pragma unroll
         for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
@@ -471,15 +471,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 128; ++c) s[c] = (c > lim) ? -INFINITY : s[c];
         }
-        float mx0 = s[0], mx1 = s[1], mx2 = s[2], mx3 = s[3];
+        // row max: four independent chains of three-input max over s[0..127]
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
 #pragma unroll
-        for (int c = 4; c < 128; c += 4) {
-          mx0 = fmaxf(mx0, s[c]);
-          mx1 = fmaxf(mx1, s[c + 1]);
-          mx2 = fmaxf(mx2, s[c + 2]);
-          mx3 = fmaxf(mx3, s[c + 3]);
+        for (int c = 0; c < 128; c += 8) {
+          mx0 = max3(mx0, s[c], s[c + 1]);
+          mx1 = max3(mx1, s[c + 2], s[c + 3]);
+          mx2 = max3(mx2, s[c + 4], s[c + 5]);
+          mx3 = max3(mx3, s[c + 6], s[c + 7]);
         }
-        const float mx = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3));
+        const float mx = fmaxf(max3(mx0, mx1, mx2), mx3);
         // The running max only moves when the tile raises it by more than
         // RESCALE_LOG2 (base 2): until then exponents stay below
         // 2^RESCALE_LOG2 and O, l and lse keep using the same stale max, so
@@ -500,10 +501,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const float a = ex2_approx(fmaf(s[32 * chunk + 2 * c], sl2, neg_m));
-            const float b = ex2_approx(fmaf(s[32 * chunk + 2 * c + 1], sl2, neg_m));
-            sum0 += a;
-            sum1 += b;
+            float x0, x1;
+            fma2(x0, x1, s[32 * chunk + 2 * c], s[32 * chunk + 2 * c + 1], sl2, sl2, neg_m, neg_m);
+            const float a = ex2_approx(x0);
+            const float b = ex2_approx(x1);
+            add2(sum0, sum1, sum0, sum1, a, b);
             pk[c] = pack2<BF16>(a, b);
           }
           tmem_st16(tS + 16 * chunk, pk);
@@ -516,9 +518,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int c0 = 0; c0 < D; c0 += 32) {
             uint32_t o[32];
             tmem_ld32(tO + c0, o);
-            tmem_wait_ld();
+            tmem_wait_ld_regs(o);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            for (int i = 0; i < 32; i += 2) {
+              float a0, a1;
+              mul2(a0, a1, __uint_as_float(o[i]), __uint_as_float(o[i + 1]), alpha, alpha);
+              o[i] = __float_as_uint(a0);
+              o[i + 1] = __float_as_uint(a1);
+            }
             tmem_st32(tO + c0, o);
           }
         }
@@ -542,7 +549,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int c0 = 0; c0 < D; c0 += 32) {
         uint32_t o[32];
         tmem_ld32(tO + c0, o);
-        tmem_wait_ld();
+        tmem_wait_ld_regs(o);
         uint32_t pk[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i)
