@@ -151,6 +151,26 @@ class ClockSampler(threading.Thread):
         return out
 
 
+def rank_seed(w, rank: int) -> int:
+    """Seed of rank ``rank``'s own copy of the workload (weak scaling: one slice per rank)."""
+    return w.seed + 1000 * rank
+
+
+def max_over_ranks(value: float, dist, device) -> float:
+    """Max of a per-rank timing over all ranks (the slowest rank sets the job time)."""
+    import torch
+    if dist is None or not dist.is_initialized() or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tflops(world: int, flops_per_step: float, steps: int, total_ms: float) -> float:
+    """Whole-job throughput: every rank ran ``steps`` steps of its own slice."""
+    return world * flops_per_step * steps / (total_ms * 1e-3) / 1e12
+
+
 def cpu_cores():
     try:
         return len(os.sched_getaffinity(0))
@@ -264,7 +284,7 @@ def main():
             dist.barrier()
 
     # each rank: its own seeded copy of the workload (weak scaling over (batch, head))
-    q, k, v = make_qkv(w.B, w.H, w.Nq, w.Nk, w.d, w.dtype, w.seed + 1000 * rank, w.qk_scale)
+    q, k, v = make_qkv(w.B, w.H, w.Nq, w.Nk, w.d, w.dtype, rank_seed(w, rank), w.qk_scale)
     qd, kd, vd = q.to(dev), k.to(dev), v.to(dev)
     od = torch.empty_like(qd)
     ld = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
@@ -298,11 +318,7 @@ def main():
     barrier()
     sampler.stop()
     kernel_ms = [e0.elapsed_time(e1) for e0, e1 in evs]
-    total_ms = sum(kernel_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(kernel_ms), dist if world > 1 else None, dev)
     st, word = attn.attn_get_device_status(sh)
     if st != 0:
         raise attn.AttnError(st, f"device status {word:#x}")
@@ -340,15 +356,11 @@ def main():
     e_end.record(stream)
     torch.cuda.synchronize()
     barrier()
-    e2e_ms = e_start.elapsed_time(e_end)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e_start.elapsed_time(e_end), dist if world > 1 else None, dev)
 
     ms_per_step = total_ms / args.steps
-    value = world * w.flops * args.steps / (total_ms * 1e-3) / 1e12
-    e2e_value = world * w.flops * args.steps / (e2e_ms * 1e-3) / 1e12
+    value = job_tflops(world, w.flops, args.steps, total_ms)
+    e2e_value = job_tflops(world, w.flops, args.steps, e2e_ms)
     per_launch_s = ms_per_step * 1e-3
     roof = roofline(w, per_launch_s, peaks)
     roof["peak_source"] = peaks["source"]

@@ -59,6 +59,12 @@ static_assert(2 * 128 * SOFTMAX_REGS + 128 * PRODUCER_REGS <= NUM_THREADS * 168,
               "register split exceeds the launch budget");
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
 constexpr float RESCALE_LOG2 = 8.0f;  // lazy-rescale threshold for the running max
+// Of every 16 key pairs in a 32-key chunk, this many take 2^x from a
+// polynomial on the FMA pipe and the rest from the MUFU ex2 unit, so the two
+// pipes share the exponentials.  At d = 64 the MUFU bounds the softmax; at
+// d = 128 the tensor core does, and the polynomial only costs issue slots.
+template <int D>
+__host__ __device__ constexpr int exp_poly_pairs() { return D == 64 ? 4 : 0; }
 
 // Device status word: 0 = healthy; otherwise 0x80000000 | site.
 __device__ unsigned int g_attn_status = 0;
@@ -471,21 +477,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 128; ++c) s[c] = (c > lim) ? -INFINITY : s[c];
         }
-        // row max: four independent chains of three-input max over s[0..127]
-        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+        // row max: eight independent chains of three-input max over s[0..127]
+        float mx[8];
 #pragma unroll
-        for (int c = 0; c < 128; c += 8) {
-          mx0 = max3(mx0, s[c], s[c + 1]);
-          mx1 = max3(mx1, s[c + 2], s[c + 3]);
-          mx2 = max3(mx2, s[c + 4], s[c + 5]);
-          mx3 = max3(mx3, s[c + 6], s[c + 7]);
+        for (int i = 0; i < 8; ++i) mx[i] = max3(s[2 * i], s[2 * i + 1], s[16 + 2 * i]);
+#pragma unroll
+        for (int c = 32; c < 128; c += 16) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], s[c + 2 * i], s[c + 2 * i + 1]);
         }
-        const float mx = fmaxf(max3(mx0, mx1, mx2), mx3);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[17 + 2 * i]);
+        const float mx_all = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]),
+                                  fmaxf(mx[6], mx[7]));
         // The running max only moves when the tile raises it by more than
         // RESCALE_LOG2 (base 2): until then exponents stay below
         // 2^RESCALE_LOG2 and O, l and lse keep using the same stale max, so
         // the result is unchanged while most O rescales are skipped.
-        const float m_cand = fmaxf(m, mx * sl2);
+        const float m_cand = fmaxf(m, mx_all * sl2);
         const bool raise = m_cand > m + RESCALE_LOG2;
         const float m_new = raise ? m_cand : m;
         const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
@@ -501,10 +510,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           uint32_t pk[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            float x0, x1;
+            float x0, x1, a, b;
             fma2(x0, x1, s[32 * chunk + 2 * c], s[32 * chunk + 2 * c + 1], sl2, sl2, neg_m, neg_m);
-            const float a = ex2_approx(x0);
-            const float b = ex2_approx(x1);
+            if (c < exp_poly_pairs<D>()) {
+              exp2_poly2(a, b, x0, x1);  // FMA pipe, in parallel with the MUFU ones
+            } else {
+              a = ex2_approx(x0);
+              b = ex2_approx(x1);
+            }
             add2(sum0, sum1, sum0, sum1, a, b);
             pk[c] = pack2<BF16>(a, b);
           }

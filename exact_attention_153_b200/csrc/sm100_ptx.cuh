@@ -288,6 +288,30 @@ __device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, f
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 
+// 2^x for a pair of fp32 values on the FMA/ALU pipes instead of the MUFU.
+// x is split as x = j + f with j = round(x) (x + 1.5 * 2^23 puts j in the
+// low mantissa bits) and f in [-1/2, 1/2]; 2^f is a degree-3 polynomial
+// (minimax in relative error, max 7.5e-5, coefficients from
+// fit_exp2_poly.py); 2^j is applied by adding j to the exponent field.  x is
+// clamped at -126 so the exponent add never underflows; results below
+// 2^-126 are returned as tiny normal or subnormal values, not zero.
+__device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
+  constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+  constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;
+  constexpr float c2 = 0.2426111251115799f, c3 = 0.0551716685295105f;
+  x0 = fmaxf(x0, -126.f);
+  x1 = fmaxf(x1, -126.f);
+  float t0, t1, j0, j1, f0, f1, p0, p1;
+  add2(t0, t1, x0, x1, kRound, kRound);
+  add2(j0, j1, t0, t1, -kRound, -kRound);
+  fma2(f0, f1, j0, j1, -1.f, -1.f, x0, x1);
+  fma2(p0, p1, c3, c3, f0, f1, c2, c2);
+  fma2(p0, p1, p0, p1, f0, f1, c1, c1);
+  fma2(p0, p1, p0, p1, f0, f1, c0, c0);
+  y0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+  y1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+}
+
 // Pack two fp32 values into one 32-bit word, `lo` in bits 0-15 and `hi` in
 // bits 16-31, rounding to nearest even.
 template <bool BF16>
