@@ -95,7 +95,8 @@ void fill_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, att
   out->grid = static_cast<int>(units < num_sms ? units : num_sms);
   out->block = NUM_THREADS;
   out->smem_bytes = d == 64 ? SmemLayout<64>::BYTES : SmemLayout<128>::BYTES;
-  out->stages = d == 64 ? SmemLayout<64>::STAGES : SmemLayout<128>::STAGES;
+  out->stages = d == 64 ? SmemLayout<64>::K_STAGES + SmemLayout<64>::V_STAGES
+                        : SmemLayout<128>::K_STAGES + SmemLayout<128>::V_STAGES;
   // score tiles per (batch, head): the same count the kernel's work units visit
   long long per_head = 0;
   for (int qt = 0; qt < q_tiles; ++qt) {

@@ -45,14 +45,15 @@ namespace attn_sm100 {
 constexpr int BLOCK_M = 128;     // query rows per Q tile (= TMEM lanes)
 constexpr int BLOCK_N = 128;     // keys per K / V tile
 // 12 warps = 3 warpgroups: two softmax warpgroups (warps 0-3, 4-7) and one
-// producer warpgroup (warp 8 issues MMAs, warp 9 issues TMA loads, warps 10-11
-// idle).  Launched at 168 registers per thread (the per-SM-sub-partition
+// producer warpgroup (warp 8 issues the S MMAs, warp 9 the TMA loads, warp 10
+// the P V MMAs, warp 11 idles).  Launched at 168 registers per thread (the per-SM-sub-partition
 // limit for 3 warps each); the producer warpgroup then gives registers up
 // and the softmax warpgroups take them: 2 * 128 * 200 + 128 * 96 = 63488 <=
 // 384 * 168, so the increase never waits on registers that do not exist.
 constexpr int NUM_THREADS = 384;
-constexpr int MMA_WARP = 8;
+constexpr int MMA_WARP = 8;    // issues S = Q K^T
 constexpr int LOAD_WARP = 9;
+constexpr int PV_WARP = 10;    // issues O += P V
 constexpr uint32_t SOFTMAX_REGS = 200;
 constexpr uint32_t PRODUCER_REGS = 96;
 static_assert(2 * 128 * SOFTMAX_REGS + 128 * PRODUCER_REGS <= NUM_THREADS * 168,
@@ -76,7 +77,7 @@ enum WaitSite : uint32_t {
   SITE_MMA_KV_FULL = 4,
   SITE_MMA_P_FULL = 5,
   SITE_SOFTMAX_S_FULL = 6,
-  SITE_SOFTMAX_O_FULL = 7,
+  SITE_SOFTMAX_O_READY = 7,
   SITE_DRAIN = 8,
 };
 
@@ -97,26 +98,40 @@ struct SmemLayout {
   static constexpr int HALF_BYTES = BLOCK_M * 64 * 2;  // one 64-column, 128-byte-swizzled slab
   static constexpr int HALVES = D / 64;
   static constexpr int TILE_BYTES = HALVES * HALF_BYTES;
-  static constexpr int STAGES = (D == 64) ? 8 : 4;
+  // separate K and V rings, filled in the order the MMA warp consumes them
+  static constexpr int K_STAGES = (D == 64) ? 4 : 2;
+  static constexpr int V_STAGES = (D == 64) ? 4 : 2;
   static constexpr int Q_OFF = 0;
-  static constexpr int KV_OFF = Q_OFF + 2 * TILE_BYTES;
-  static constexpr int BAR_OFF = KV_OFF + STAGES * TILE_BYTES;
+  static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
+  static constexpr int V_OFF = K_OFF + K_STAGES * TILE_BYTES;
+  static constexpr int BAR_OFF = V_OFF + V_STAGES * TILE_BYTES;
+  // S/P buffers in TMEM: three at d = 64 (so a tile's next S is computed
+  // while its current P is still being written), two at d = 128 (TMEM holds
+  // 2 x 128 S columns + 2 x 128 O columns and nothing more).
+  static constexpr int NSB = (D == 64) ? 3 : 2;
   // mbarrier indices
-  static constexpr int KV_FULL = 0;
-  static constexpr int KV_EMPTY = STAGES;
-  static constexpr int Q_FULL = 2 * STAGES;
-  static constexpr int Q_EMPTY = 2 * STAGES + 1;
-  static constexpr int S_FULL = 2 * STAGES + 2;  // + tile
-  static constexpr int P_FULL = 2 * STAGES + 4;  // + tile
-  static constexpr int O_FULL = 2 * STAGES + 6;  // + tile
-  static constexpr int DRAIN = 2 * STAGES + 8;
-  static constexpr int NUM_BARS = 2 * STAGES + 9;
+  static constexpr int K_FULL = 0;
+  static constexpr int K_EMPTY = K_FULL + K_STAGES;
+  static constexpr int V_FULL = K_EMPTY + K_STAGES;
+  static constexpr int V_EMPTY = V_FULL + V_STAGES;
+  static constexpr int Q_FULL = V_EMPTY + V_STAGES;
+  static constexpr int Q_EMPTY = Q_FULL + 1;
+  // S ready: one barrier per (buffer, tile), so each softmax warpgroup only
+  // waits on phases it alone consumes (a per-buffer barrier shared by both
+  // tiles could be two phases behind a warpgroup that skipped an item).
+  static constexpr int S_FULL = Q_EMPTY + 1;       // + 2 * buffer + tile
+  static constexpr int P_FULL = S_FULL + 2 * NSB;  // + buffer (one waiter: the MMA warp)
+  static constexpr int O_READY = P_FULL + NSB; // + tile: one phase per P V MMA of the tile
+  static constexpr int PV_DONE = O_READY + 2;  // + buffer: P V of that buffer finished
+  static constexpr int DRAIN = PV_DONE + NSB;  // + 0 (S warp), + 1 (P V warp)
+  static constexpr int NUM_BARS = DRAIN + 2;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // TMEM address, abort flag
   static constexpr int BYTES = MISC_OFF + 16 + 1024;      // + slack to align the base to 1 KB
-  // TMEM columns (512 allocated): S/P of tile 0 and 1, then O of tile 0 and 1
+  // TMEM columns (512 allocated): S/P buffers, then O of tile 0 and tile 1
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t S_COL = 0;    // + 128 * tile
-  static constexpr uint32_t O_COL = 256;  // + D * tile
+  static constexpr uint32_t S_COL = 0;           // + 128 * buffer
+  static constexpr uint32_t O_COL = 128 * NSB;   // + D * tile
+  static_assert(O_COL + 2 * D <= TMEM_COLS, "TMEM budget");
 };
 
 struct Unit {
@@ -170,6 +185,29 @@ __device__ __forceinline__ Unit decode_item(const FwdParams& p, int u, int item)
   return w;
 }
 
+// The S sequence of one item: the MMA warp computes the score tiles of the
+// two Q tiles alternately, S_0(0), S_1(0), S_0(1), S_1(1), ..., and, when
+// one tile visits one more K/V tile than the other, the longer tile's last
+// one at the end.  Position k of that sequence goes to S/P buffer
+// (k_item_base + k) % NSB.
+struct SeqPos {
+  int t, j;
+};
+__device__ __forceinline__ SeqPos seq_at(const Unit& w, int k) {
+  const int m = min(w.n[0], w.n[1]);
+  if (k < 2 * m) return {k & 1, k >> 1};
+  return {w.n[0] > w.n[1] ? 0 : 1, m + (k - 2 * m)};
+}
+__device__ __forceinline__ int seq_pos(const Unit& w, int t, int j) {
+  const int m = min(w.n[0], w.n[1]);
+  return j < m ? 2 * j + t : 2 * m + (j - m);
+}
+// K_j / V_j is used for the last time by tile 1, or by tile 0 when tile 1
+// does not visit j.
+__device__ __forceinline__ bool last_use(const Unit& w, SeqPos s) {
+  return s.t == 1 || s.j >= w.n[1];
+}
+
 // Bounded wait on one mbarrier phase, fully inlined (a call here would make
 // the compiler save live registers to local memory on every slow wait).
 // Returns false on timeout (status word set, abort flag raised) or, when
@@ -199,6 +237,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using L = SmemLayout<D>;
+  constexpr int NSB = L::NSB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -210,18 +249,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto bar = [&](int i) -> uint32_t { return sbase + L::BAR_OFF + 8u * i; };
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < L::STAGES; ++s) {
-      mbar_init(bar(L::KV_FULL + s), 1);
-      mbar_init(bar(L::KV_EMPTY + s), 1);
+    for (int s = 0; s < L::K_STAGES; ++s) {
+      mbar_init(bar(L::K_FULL + s), 1);
+      mbar_init(bar(L::K_EMPTY + s), 1);
+    }
+    for (int s = 0; s < L::V_STAGES; ++s) {
+      mbar_init(bar(L::V_FULL + s), 1);
+      mbar_init(bar(L::V_EMPTY + s), 1);
     }
     mbar_init(bar(L::Q_FULL), 1);
     mbar_init(bar(L::Q_EMPTY), 1);
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(bar(L::S_FULL + t), 1);
-      mbar_init(bar(L::P_FULL + t), 4 * 32);
-      mbar_init(bar(L::O_FULL + t), 1);
+    for (int b = 0; b < NSB; ++b) {
+      mbar_init(bar(L::S_FULL + 2 * b), 1);
+      mbar_init(bar(L::S_FULL + 2 * b + 1), 1);
+      mbar_init(bar(L::P_FULL + b), 4 * 32);
     }
-    mbar_init(bar(L::DRAIN), 1);
+    mbar_init(bar(L::O_READY + 0), 1);
+    mbar_init(bar(L::O_READY + 1), 1);
+    for (int b = 0; b < NSB; ++b) mbar_init(bar(L::PV_DONE + b), 1);
+    mbar_init(bar(L::DRAIN + 0), 1);
+    mbar_init(bar(L::DRAIN + 1), 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -248,21 +295,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // registers before every MMA, which made the issue the bottleneck).
     const bool leader = elect_one();
     const uint32_t q_smem = sbase + L::Q_OFF;
-    const uint32_t kv_smem = sbase + L::KV_OFF;
+    const uint32_t k_smem = sbase + L::K_OFF;
+    const uint32_t v_smem = sbase + L::V_OFF;
     auto warp_wait = [&](uint32_t b, uint32_t parity, uint32_t site) -> bool {
       const bool r = wait_phase(b, parity, abort_flag, site);
       return __all_sync(0xffffffffu, r);
     };
     if (warp == LOAD_WARP) {
       // ----------------------------------------------------------- TMA producer
-      uint32_t kv_it = 0, units = 0;
+      // K_j and V_j are loaded in exactly the order the MMA warp first needs
+      // them (the same walk over the S sequence), each into its own ring.
+      uint32_t kpos = 0, vpos = 0, items_done = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
         const int items = unit_items(p, u);
         for (int item = 0; ok && item < items; ++item) {
           const Unit w = decode_item(p, u, item);
-          if (units > 0) {
-            ok = warp_wait(bar(L::Q_EMPTY), (units - 1) & 1, SITE_LOAD_Q_EMPTY);
+          if (items_done > 0) {
+            ok = warp_wait(bar(L::Q_EMPTY), (items_done - 1) & 1, SITE_LOAD_Q_EMPTY);
             if (!ok) break;
           }
           if (leader) {
@@ -275,162 +325,251 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                             h * 64, w.q0 + t * BLOCK_M, w.bh);
           }
           __syncwarp();
-          ++units;
-          for (int j = 0; ok && j < w.nmax; ++j) {
-#pragma unroll
-            for (int which = 0; which < 2; ++which) {
-              const uint32_t st = kv_it % L::STAGES;
-              const uint32_t ph = (kv_it / L::STAGES) & 1;
-              if (kv_it >= static_cast<uint32_t>(L::STAGES)) {
-                ok = warp_wait(bar(L::KV_EMPTY + st), ph ^ 1, SITE_LOAD_KV_EMPTY);
-                if (!ok) break;
-              }
+          ++items_done;
+          int k_next = 0, v_next = 0;
+          auto load_k_upto = [&](int j) -> bool {
+            for (; k_next <= j; ++k_next) {
+              const uint32_t st = kpos % L::K_STAGES, ph = (kpos / L::K_STAGES) & 1;
+              if (kpos >= static_cast<uint32_t>(L::K_STAGES) &&
+                  !warp_wait(bar(L::K_EMPTY + st), ph ^ 1, SITE_LOAD_KV_EMPTY))
+                return false;
               if (leader) {
-                mbar_arrive_expect_tx(bar(L::KV_FULL + st), L::TILE_BYTES);
+                mbar_arrive_expect_tx(bar(L::K_FULL + st), L::TILE_BYTES);
 #pragma unroll
                 for (int h = 0; h < L::HALVES; ++h)
-                  tma_load_3d(kv_smem + st * L::TILE_BYTES + h * L::HALF_BYTES,
-                              which ? &tm_v : &tm_k, bar(L::KV_FULL + st), h * 64, j * BLOCK_N,
-                              w.bh);
+                  tma_load_3d(k_smem + st * L::TILE_BYTES + h * L::HALF_BYTES, &tm_k,
+                              bar(L::K_FULL + st), h * 64, k_next * BLOCK_N, w.bh);
               }
               __syncwarp();
-              ++kv_it;
+              ++kpos;
             }
+            return true;
+          };
+          auto load_v_upto = [&](int j) -> bool {
+            for (; v_next <= j; ++v_next) {
+              const uint32_t st = vpos % L::V_STAGES, ph = (vpos / L::V_STAGES) & 1;
+              if (vpos >= static_cast<uint32_t>(L::V_STAGES) &&
+                  !warp_wait(bar(L::V_EMPTY + st), ph ^ 1, SITE_LOAD_KV_EMPTY))
+                return false;
+              if (leader) {
+                mbar_arrive_expect_tx(bar(L::V_FULL + st), L::TILE_BYTES);
+#pragma unroll
+                for (int h = 0; h < L::HALVES; ++h)
+                  tma_load_3d(v_smem + st * L::TILE_BYTES + h * L::HALF_BYTES, &tm_v,
+                              bar(L::V_FULL + st), h * 64, v_next * BLOCK_N, w.bh);
+              }
+              __syncwarp();
+              ++vpos;
+            }
+            return true;
+          };
+          const int total = w.n[0] + w.n[1];
+          for (int k = 0; ok && k < min(NSB, total); ++k) ok = load_k_upto(seq_at(w, k).j);
+          for (int k = 0; ok && k < total; ++k) {
+            ok = load_v_upto(seq_at(w, k).j);
+            if (ok && k + NSB < total) ok = load_k_upto(seq_at(w, k + NSB).j);
           }
         }
       }
       // Every issued load must have landed before the CTA may exit.
-      const uint32_t first = kv_it > static_cast<uint32_t>(L::STAGES) ? kv_it - L::STAGES : 0;
-      for (uint32_t i = first; i < kv_it; ++i)
-        wait_phase(bar(L::KV_FULL + i % L::STAGES), (i / L::STAGES) & 1, abort_flag, SITE_DRAIN,
+      for (uint32_t i = kpos > L::K_STAGES ? kpos - L::K_STAGES : 0; i < kpos; ++i)
+        wait_phase(bar(L::K_FULL + i % L::K_STAGES), (i / L::K_STAGES) & 1, abort_flag, SITE_DRAIN,
                    false);
-      if (units > 0) wait_phase(bar(L::Q_FULL), (units - 1) & 1, abort_flag, SITE_DRAIN, false);
+      for (uint32_t i = vpos > L::V_STAGES ? vpos - L::V_STAGES : 0; i < vpos; ++i)
+        wait_phase(bar(L::V_FULL + i % L::V_STAGES), (i / L::V_STAGES) & 1, abort_flag, SITE_DRAIN,
+                   false);
+      if (items_done > 0)
+        wait_phase(bar(L::Q_FULL), (items_done - 1) & 1, abort_flag, SITE_DRAIN, false);
       __syncwarp();
-    } else if (warp == MMA_WARP) {
-      // ----------------------------------------------------------- MMA issuer
+    } else if (warp == MMA_WARP || warp == PV_WARP) {
+      // ----------------------------------------------------------- MMA issuers
+      // Two warps feed the tensor core.  Warp 8 issues S(g) = Q_t K_j^T for
+      // the g-th score tile of the CTA into S/P buffer g % NSB as soon as
+      // its K tile is loaded and the P V that last read that buffer is done;
+      // it can therefore run up to NSB tiles ahead of the softmax.  Warp 10
+      // issues O_t += P(g) V_j as soon as the softmax has written P(g).  Each
+      // warp only waits on its own inputs, so one waiting for the softmax
+      // does not hold back the other's work.
       constexpr uint32_t IDESC_S = idesc_f16(BF16, false, false, BLOCK_M, BLOCK_N);
       constexpr uint32_t IDESC_O = idesc_f16(BF16, false, true, BLOCK_M, D);
-      // S_t = Q_t K^T: both operands K-major (head dim contiguous), 128-byte
-      // swizzle, 8-row groups 1024 bytes apart; each k-step covers 16
-      // elements = 32 bytes of a 128-byte row, the head dim > 64 continues in
-      // the next 16 KB slab.  Descriptors are built once; a k-step or a ring
-      // slot only adds (byte offset >> 4) to the start-address field (every
-      // address stays below 256 KB, so the add never carries out of it).
+      // S: both operands K-major (head dim contiguous), 128-byte swizzle,
+      // 8-row groups 1024 bytes apart; each k-step covers 16 elements = 32
+      // bytes of a 128-byte row, the head dim > 64 continues in the next 16 KB
+      // slab.  Descriptors are built once; a k-step or a ring slot only adds
+      // (byte offset >> 4) to the start-address field (every address stays
+      // below 256 KB, so the add never carries out of it).
       const uint64_t q_desc = sw128_desc(q_smem, 16, 1024);
-      const uint64_t k_desc = sw128_desc(kv_smem, 16, 1024);
-      // O_t += P_t V: P from TMEM (16 keys = 8 columns per k-step), V
-      // MN-major (head dim contiguous): 8-key groups 1024 bytes apart,
-      // 64-column slabs 16 KB apart; each k-step advances 16 keys = 2 KB.
-      const uint64_t v_desc = sw128_desc(kv_smem, L::HALF_BYTES, 1024);
+      const uint64_t k_desc = sw128_desc(k_smem, 16, 1024);
+      // P V: P from TMEM (16 keys = 8 columns per k-step), V MN-major (head
+      // dim contiguous): 8-key groups 1024 bytes apart, 64-column slabs 16 KB
+      // apart; each k-step advances 16 keys = 2 KB.
+      const uint64_t v_desc = sw128_desc(v_smem, L::HALF_BYTES, 1024);
       const uint32_t tmem_s = tmem_base + L::S_COL;
       const uint32_t tmem_o = tmem_base + L::O_COL;
+      // With only two S/P buffers (d = 128) the next S of a tile must reuse
+      // the buffer its last P V reads; one thread issuing both keeps them in
+      // order in the tensor pipe without waiting for the P V to finish, so
+      // at d = 128 warp 8 issues everything in sequence order (P V(g), then
+      // S(g + 2)) and warp 10 idles.
+      constexpr bool kSplit = (NSB > 2);
+      if (!kSplit && warp == PV_WARP) {
+        // nothing to do
+      } else {
+      const bool is_s = (warp == MMA_WARP);
 
-      auto issue_s = [&](int t, uint32_t stage) {
-        const uint64_t a = q_desc + static_cast<uint32_t>(t * (L::TILE_BYTES >> 4));
-        const uint64_t b = k_desc + stage * static_cast<uint32_t>(L::TILE_BYTES >> 4);
-        if (leader) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = ((kk / 4) * L::HALF_BYTES + (kk % 4) * 32) >> 4;
-            mma_ss(tmem_s + 128 * t, a + off, b + off, IDESC_S, kk > 0 ? 1u : 0u);
-          }
-        }
-      };
-      auto issue_pv = [&](int t, uint32_t stage, bool accumulate) {
-        const uint64_t b = v_desc + stage * static_cast<uint32_t>(L::TILE_BYTES >> 4);
-        if (leader) {
-#pragma unroll
-          for (int kk = 0; kk < BLOCK_N / 16; ++kk)
-            mma_ts(tmem_o + D * t, tmem_s + 128 * t + kk * 8, b + kk * (2048 >> 4), IDESC_O,
-                   (accumulate || kk > 0) ? 1u : 0u);
-        }
-      };
-      auto commit = [&](uint32_t b) {
-        if (leader) mma_commit(b);
-      };
-
-      uint32_t kv_it = 0, q_phase = 0;
-      uint32_t p_phase[2] = {0, 0};
+      uint32_t pos = 0, g = 0, q_phase = 0;  // ring position of K_0 / V_0 of the item; score tile count
+      uint32_t buf = 0, round = 0;           // g % NSB, g / NSB
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
         const int items = unit_items(p, u);
         for (int item = 0; ok && item < items; ++item) {
           const Unit w = decode_item(p, u, item);
-          ok = warp_wait(bar(L::Q_FULL), q_phase, SITE_MMA_Q_FULL);
-          if (!ok) break;
-          q_phase ^= 1;
-          {
-            const uint32_t st = kv_it % L::STAGES, ph = (kv_it / L::STAGES) & 1;
-            ++kv_it;
-            ok = warp_wait(bar(L::KV_FULL + st), ph, SITE_MMA_KV_FULL);
+          const int total = w.n[0] + w.n[1];
+          if (is_s) {
+            ok = warp_wait(bar(L::Q_FULL), q_phase, SITE_MMA_Q_FULL);
             if (!ok) break;
-            tc_fence_after();
-#pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              if (w.n[t] > 0) {
-                issue_s(t, st);
-                commit(bar(L::S_FULL + t));
-              }
-            }
-            commit(bar(L::KV_EMPTY + st));
-            __syncwarp();
+            q_phase ^= 1;
           }
-          for (int j = 0; ok && j < w.nmax; ++j) {
-            const uint32_t vst = kv_it % L::STAGES, vph = (kv_it / L::STAGES) & 1;
-            ++kv_it;
-            const bool has_next = j + 1 < w.nmax;
-            uint32_t kst = 0, kph = 0;
-            if (has_next) {
-              kst = kv_it % L::STAGES;
-              kph = (kv_it / L::STAGES) & 1;
-              ++kv_it;
-            }
-            ok = warp_wait(bar(L::KV_FULL + vst), vph, SITE_MMA_KV_FULL);
-            if (!ok) break;
-            bool k_ready = false;
+          int ready_j = -1;
+          if constexpr (!kSplit) {
+            // in-order issue: S(0), S(1), then P V(k) followed by S(k + 2)
+            int k_ready = -1, v_ready = -1;
+            auto issue_s = [&](int k) -> bool {
+              const SeqPos sp = seq_at(w, k);
+              const uint32_t kp = pos + sp.j;
+              const uint32_t st = kp % L::K_STAGES;
+              if (sp.j > k_ready) {
+                if (!warp_wait(bar(L::K_FULL + st), (kp / L::K_STAGES) & 1, SITE_MMA_KV_FULL))
+                  return false;
+                tc_fence_after();
+                k_ready = sp.j;
+              }
+              const uint32_t b = (g + k) % NSB;
+              const uint64_t a = q_desc + static_cast<uint32_t>(sp.t * (L::TILE_BYTES >> 4));
+              const uint64_t bd = k_desc + st * static_cast<uint32_t>(L::TILE_BYTES >> 4);
+              if (leader) {
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-              if (!ok || j >= w.n[t]) continue;
-              ok = warp_wait(bar(L::P_FULL + t), p_phase[t], SITE_MMA_P_FULL);
-              if (!ok) continue;
-              p_phase[t] ^= 1;
-              tc_fence_after();
-              issue_pv(t, vst, j > 0);
-              if (j + 1 < w.n[t]) {
-                if (!k_ready) {
-                  ok = warp_wait(bar(L::KV_FULL + kst), kph, SITE_MMA_KV_FULL);
-                  if (!ok) continue;
-                  tc_fence_after();
-                  k_ready = true;
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const uint32_t off = ((kk / 4) * L::HALF_BYTES + (kk % 4) * 32) >> 4;
+                  mma_ss(tmem_s + 128 * b, a + off, bd + off, IDESC_S, kk > 0 ? 1u : 0u);
                 }
-                issue_s(t, kst);
-                commit(bar(L::S_FULL + t));
-              } else {
-                commit(bar(L::O_FULL + t));
+                mma_commit(bar(L::S_FULL + 2 * b + sp.t));
+                if (last_use(w, sp)) mma_commit(bar(L::K_EMPTY + st));
               }
-              __syncwarp();
-            }
-            if (!ok) break;
-            commit(bar(L::KV_EMPTY + vst));
-            if (has_next) {
-              if (!k_ready) {
-                ok = warp_wait(bar(L::KV_FULL + kst), kph, SITE_MMA_KV_FULL);
-                if (!ok) break;
+              return true;
+            };
+            for (int k = 0; ok && k < min(NSB, total); ++k) ok = issue_s(k);
+            for (int k = 0; ok && k < total; ++k) {
+              const SeqPos sp = seq_at(w, k);
+              const uint32_t vp = pos + sp.j;
+              const uint32_t st = vp % L::V_STAGES;
+              if (sp.j > v_ready) {
+                if (!warp_wait(bar(L::V_FULL + st), (vp / L::V_STAGES) & 1, SITE_MMA_KV_FULL)) {
+                  ok = false;
+                  break;
+                }
+                v_ready = sp.j;
               }
-              commit(bar(L::KV_EMPTY + kst));
+              const uint32_t gk = g + k;
+              const uint32_t b = gk % NSB;
+              if (!warp_wait(bar(L::P_FULL + b), (gk / NSB) & 1, SITE_MMA_P_FULL)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint64_t bd = v_desc + st * static_cast<uint32_t>(L::TILE_BYTES >> 4);
+              if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < BLOCK_N / 16; ++kk)
+                  mma_ts(tmem_o + D * sp.t, tmem_s + 128 * b + kk * 8, bd + kk * (2048 >> 4),
+                         IDESC_O, (sp.j > 0 || kk > 0) ? 1u : 0u);
+                // in-order issue: S_t(j + 1) completing already implies this
+                // P V completed, so only the tile's last P V is signalled
+                if (sp.j + 1 == (sp.t ? w.n[1] : w.n[0])) mma_commit(bar(L::O_READY + sp.t));
+                if (last_use(w, sp)) mma_commit(bar(L::V_EMPTY + st));
+              }
+              // the buffer of P(k) is refilled by S(k + NSB): same thread, so
+              // the tensor pipe runs it after this P V
+              if (k + NSB < total) ok = issue_s(k + NSB);
             }
-            __syncwarp();
+            g += total;
+          } else
+          for (int k = 0; k < total; ++k) {
+            const SeqPos sp = seq_at(w, k);
+            if (is_s) {
+              const uint32_t kp = pos + sp.j;
+              const uint32_t st = kp % L::K_STAGES;
+              if (sp.j > ready_j) {
+                if (!warp_wait(bar(L::K_FULL + st), (kp / L::K_STAGES) & 1, SITE_MMA_KV_FULL)) {
+                  ok = false;
+                  break;
+                }
+                ready_j = sp.j;
+              }
+              if (g >= static_cast<uint32_t>(NSB) &&
+                  !warp_wait(bar(L::PV_DONE + buf), (round - 1) & 1, SITE_MMA_P_FULL)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint64_t a = q_desc + static_cast<uint32_t>(sp.t * (L::TILE_BYTES >> 4));
+              const uint64_t bd = k_desc + st * static_cast<uint32_t>(L::TILE_BYTES >> 4);
+              if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                  const uint32_t off = ((kk / 4) * L::HALF_BYTES + (kk % 4) * 32) >> 4;
+                  mma_ss(tmem_s + 128 * buf, a + off, bd + off, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(bar(L::S_FULL + 2 * buf + sp.t));
+                if (last_use(w, sp)) mma_commit(bar(L::K_EMPTY + st));
+              }
+            } else {
+              const uint32_t vp = pos + sp.j;
+              const uint32_t st = vp % L::V_STAGES;
+              if (sp.j > ready_j) {
+                if (!warp_wait(bar(L::V_FULL + st), (vp / L::V_STAGES) & 1, SITE_MMA_KV_FULL)) {
+                  ok = false;
+                  break;
+                }
+                ready_j = sp.j;
+              }
+              if (!warp_wait(bar(L::P_FULL + buf), round & 1, SITE_MMA_P_FULL)) {
+                ok = false;
+                break;
+              }
+              tc_fence_after();
+              const uint64_t bd = v_desc + st * static_cast<uint32_t>(L::TILE_BYTES >> 4);
+              if (leader) {
+#pragma unroll
+                for (int kk = 0; kk < BLOCK_N / 16; ++kk)
+                  mma_ts(tmem_o + D * sp.t, tmem_s + 128 * buf + kk * 8, bd + kk * (2048 >> 4),
+                         IDESC_O, (sp.j > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(bar(L::O_READY + sp.t));
+                mma_commit(bar(L::PV_DONE + buf));
+                if (last_use(w, sp)) mma_commit(bar(L::V_EMPTY + st));
+              }
+            }
+            ++g;
+            if (++buf == static_cast<uint32_t>(NSB)) {
+              buf = 0;
+              ++round;
+            }
           }
           if (!ok) break;
-          commit(bar(L::Q_EMPTY));
+          // every S of the item has been issued: the Q tiles may be replaced
+          // once those MMAs complete
+          if (is_s && leader) mma_commit(bar(L::Q_EMPTY));
           __syncwarp();
+          pos += w.nmax;
         }
       }
       // All MMAs (and their commits) must be finished before TMEM is freed.
-      commit(bar(L::DRAIN));
+      const uint32_t drain = bar(L::DRAIN + (is_s ? 0 : 1));
+      if (leader) mma_commit(drain);
       __syncwarp();
-      wait_phase(bar(L::DRAIN), 0, abort_flag, SITE_DRAIN, false);
+      wait_phase(drain, 0, abort_flag, SITE_DRAIN, false);
       __syncwarp();
+      }
     }
   } else {
     regs_increase<SOFTMAX_REGS>();
@@ -439,144 +578,163 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int quarter = warp % 4;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem_base + lane_off + L::S_COL + 128 * t;
+    const uint32_t tS0 = tmem_base + lane_off + L::S_COL;
     const uint32_t tO = tmem_base + lane_off + L::O_COL + D * t;
     const float sl2 = p.scale_log2;
-    uint32_t s_phase = 0, o_phase = 0;
+    uint32_t o_phase = 0, sk = 0;
+    uint32_t s_parity = 0;  // bit b: parity of the next S_FULL(b, t) phase this warpgroup waits for
     bool ok = true;
     for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-     const int items = unit_items(p, u);
-     for (int item = 0; ok && item < items; ++item) {
-      const Unit w = decode_item(p, u, item);
-      const int n = t ? w.n[1] : w.n[0];
-      if (n == 0) continue;
-      const int q_start = w.q0 + t * BLOCK_M;
-      const int row = q_start + r;
-      // last key this row may see (top-left causal: key j <= query i)
-      const int last_key = p.causal ? min(p.Nk - 1, row) : (p.Nk - 1);
-      float m = -INFINITY, l = 0.f;
-      for (int j = 0; j < n; ++j) {
-        ok = wait_phase(bar(L::S_FULL + t), s_phase, abort_flag, SITE_SOFTMAX_S_FULL);
+      const int items = unit_items(p, u);
+      for (int item = 0; ok && item < items; ++item) {
+        const Unit w = decode_item(p, u, item);
+        const int n = t ? w.n[1] : w.n[0];
+        const uint32_t item_sk = sk;
+        sk += w.n[0] + w.n[1];
+        if (n == 0) continue;
+        const int q_start = w.q0 + t * BLOCK_M;
+        const int row = q_start + r;
+        // last key this row may see (top-left causal: key j <= query i)
+        const int last_key = p.causal ? min(p.Nk - 1, row) : (p.Nk - 1);
+        float m = -INFINITY, l = 0.f;
+        for (int j = 0; j < n; ++j) {
+          const uint32_t kg = item_sk + seq_pos(w, t, j);
+          const uint32_t b = kg % NSB;
+          const uint32_t tS = tS0 + 128 * b;
+          ok = wait_phase(bar(L::S_FULL + 2 * b + t), (s_parity >> b) & 1u, abort_flag,
+                          SITE_SOFTMAX_S_FULL);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          s_parity ^= 1u << b;
+          tc_fence_after();
+          uint32_t sr[128];
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * c));
+          tmem_wait_ld_regs(sr);
+          float s[128];
+#pragma unroll
+          for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+
+          const int k0 = j * BLOCK_N;
+          const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > q_start);
+          if (need_mask) {
+            const int lim = last_key - k0;  // columns > lim are masked
+#pragma unroll
+            for (int c = 0; c < 128; ++c) s[c] = (c > lim) ? -INFINITY : s[c];
+          }
+          // row max: eight independent chains of three-input max over s[0..127]
+          float mx[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = max3(s[2 * i], s[2 * i + 1], s[16 + 2 * i]);
+#pragma unroll
+          for (int c = 32; c < 128; c += 16) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], s[c + 2 * i], s[c + 2 * i + 1]);
+          }
+#pragma unroll
+          for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[17 + 2 * i]);
+          const float mx_all = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]),
+                                    fmaxf(mx[6], mx[7]));
+          // The running max only moves when the tile raises it by more than
+          // RESCALE_LOG2 (base 2): until then exponents stay below
+          // 2^RESCALE_LOG2 and O, l and lse keep using the same stale max, so
+          // the result is unchanged while most O rescales are skipped.
+          const float m_cand = fmaxf(m, mx_all * sl2);
+          const bool raise = m_cand > m + RESCALE_LOG2;
+          const float m_new = raise ? m_cand : m;
+          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+          const float alpha = raise ? ex2_approx(m - m_use) : 1.f;
+          const float neg_m = -m_use;
+
+          // P = 2^(s * scale * log2 e - m), packed two keys per 32-bit TMEM
+          // column (even key in the low half), written over S in 16-column
+          // chunks so each chunk's S registers die as it is stored.
+          float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+          for (int chunk = 0; chunk < 4; ++chunk) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int c = 0; c < 16; ++c) {
+              float x0, x1, a, bb;
+              fma2(x0, x1, s[32 * chunk + 2 * c], s[32 * chunk + 2 * c + 1], sl2, sl2, neg_m, neg_m);
+              if (c < exp_poly_pairs<D>()) {
+                exp2_poly2(a, bb, x0, x1);  // FMA pipe, in parallel with the MUFU ones
+              } else {
+                a = ex2_approx(x0);
+                bb = ex2_approx(x1);
+              }
+              add2(sum0, sum1, sum0, sum1, a, bb);
+              pk[c] = pack2<BF16>(a, bb);
+            }
+            tmem_st16(tS + 16 * chunk, pk);
+          }
+          l = l * alpha + (sum0 + sum1);
+          m = m_new;
+
+          // O_t may only be touched once the previous P V of this tile is
+          // done: with split issue that is its own signal; with in-order issue
+          // (two S buffers) the S just read was queued behind that P V.
+          if (j > 0) {
+            if constexpr (NSB > 2) {
+              ok = wait_phase(bar(L::O_READY + t), o_phase, abort_flag, SITE_SOFTMAX_O_READY);
+              ok = __all_sync(0xffffffffu, ok);
+              if (!ok) break;
+              o_phase ^= 1;
+              tc_fence_after();
+            }
+            if (__any_sync(0xffffffffu, raise)) {
+#pragma unroll
+              for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                tmem_ld32(tO + c0, o);
+                tmem_wait_ld_regs(o);
+#pragma unroll
+                for (int i = 0; i < 32; i += 2) {
+                  float a0, a1;
+                  mul2(a0, a1, __uint_as_float(o[i]), __uint_as_float(o[i + 1]), alpha, alpha);
+                  o[i] = __float_as_uint(a0);
+                  o[i + 1] = __float_as_uint(a1);
+                }
+                tmem_st32(tO + c0, o);
+              }
+            }
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(bar(L::P_FULL + b));
+        }
+        if (!ok) break;
+
+        // --------------------------------------------------------- epilogue
+        ok = wait_phase(bar(L::O_READY + t), o_phase, abort_flag, SITE_SOFTMAX_O_READY);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
-        s_phase ^= 1;
+        o_phase ^= 1;
         tc_fence_after();
-        uint32_t sr[128];
+        const float inv_l = 1.f / l;
+        const bool in_range = row < p.Nq;
+        uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
+                                               (static_cast<size_t>(w.bh) * p.Nq + row) * D);
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * c));
-        tmem_wait_ld_regs(sr);
-        float s[128];
-#pragma unroll
-        for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-
-        const int k0 = j * BLOCK_N;
-        const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > q_start);
-        if (need_mask) {
-          const int lim = last_key - k0;  // columns > lim are masked
-#pragma unroll
-          for (int c = 0; c < 128; ++c) s[c] = (c > lim) ? -INFINITY : s[c];
-        }
-        // row max: eight independent chains of three-input max over s[0..127]
-        float mx[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = max3(s[2 * i], s[2 * i + 1], s[16 + 2 * i]);
-#pragma unroll
-        for (int c = 32; c < 128; c += 16) {
-#pragma unroll
-          for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], s[c + 2 * i], s[c + 2 * i + 1]);
-        }
-#pragma unroll
-        for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[17 + 2 * i]);
-        const float mx_all = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]),
-                                  fmaxf(mx[6], mx[7]));
-        // The running max only moves when the tile raises it by more than
-        // RESCALE_LOG2 (base 2): until then exponents stay below
-        // 2^RESCALE_LOG2 and O, l and lse keep using the same stale max, so
-        // the result is unchanged while most O rescales are skipped.
-        const float m_cand = fmaxf(m, mx_all * sl2);
-        const bool raise = m_cand > m + RESCALE_LOG2;
-        const float m_new = raise ? m_cand : m;
-        const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-        const float alpha = raise ? ex2_approx(m - m_use) : 1.f;
-        const float neg_m = -m_use;
-
-        // P = 2^(s * scale * log2 e - m), packed two keys per 32-bit TMEM
-        // column (even key in the low half), written over S in 16-column
-        // chunks so each chunk's S registers die as it is stored.
-        float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-        for (int chunk = 0; chunk < 4; ++chunk) {
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tO + c0, o);
+          tmem_wait_ld_regs(o);
           uint32_t pk[16];
 #pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            float x0, x1, a, b;
-            fma2(x0, x1, s[32 * chunk + 2 * c], s[32 * chunk + 2 * c + 1], sl2, sl2, neg_m, neg_m);
-            if (c < exp_poly_pairs<D>()) {
-              exp2_poly2(a, b, x0, x1);  // FMA pipe, in parallel with the MUFU ones
-            } else {
-              a = ex2_approx(x0);
-              b = ex2_approx(x1);
-            }
-            add2(sum0, sum1, sum0, sum1, a, b);
-            pk[c] = pack2<BF16>(a, b);
-          }
-          tmem_st16(tS + 16 * chunk, pk);
-        }
-        l = l * alpha + (sum0 + sum1);
-        m = m_new;
-
-        if (__any_sync(0xffffffffu, raise && j > 0)) {
+          for (int i = 0; i < 16; ++i)
+            pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
+          if (in_range) {
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tO + c0, o);
-            tmem_wait_ld_regs(o);
-#pragma unroll
-            for (int i = 0; i < 32; i += 2) {
-              float a0, a1;
-              mul2(a0, a1, __uint_as_float(o[i]), __uint_as_float(o[i + 1]), alpha, alpha);
-              o[i] = __float_as_uint(a0);
-              o[i + 1] = __float_as_uint(a1);
-            }
-            tmem_st32(tO + c0, o);
+            for (int v4 = 0; v4 < 4; ++v4)
+              orow[c0 / 8 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
           }
         }
-        tmem_wait_st();
+        if (p.lse != nullptr && in_range)
+          p.lse[static_cast<size_t>(w.bh) * p.Nq + row] = (m + lg2_approx(l)) * 0.69314718055994531f;
         tc_fence_before();
-        mbar_arrive(bar(L::P_FULL + t));
       }
-      if (!ok) break;
-
-      // ----------------------------------------------------------- epilogue
-      ok = wait_phase(bar(L::O_FULL + t), o_phase, abort_flag, SITE_SOFTMAX_O_FULL);
-      ok = __all_sync(0xffffffffu, ok);
-      if (!ok) break;
-      o_phase ^= 1;
-      tc_fence_after();
-      const float inv_l = 1.f / l;
-      const bool in_range = row < p.Nq;
-      uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
-                                             (static_cast<size_t>(w.bh) * p.Nq + row) * D);
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        tmem_ld32(tO + c0, o);
-        tmem_wait_ld_regs(o);
-        uint32_t pk[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i)
-          pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-        if (in_range) {
-#pragma unroll
-          for (int v4 = 0; v4 < 4; ++v4)
-            orow[c0 / 8 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
-        }
-      }
-      if (p.lse != nullptr && in_range)
-        p.lse[static_cast<size_t>(w.bh) * p.Nq + row] = (m + lg2_approx(l)) * 0.69314718055994531f;
-      tc_fence_before();
-     }
     }
   }
 
