@@ -45,15 +45,16 @@ namespace attn_sm100 {
 constexpr int BLOCK_M = 128;     // query rows per Q tile (= TMEM lanes)
 constexpr int BLOCK_N = 128;     // keys per K / V tile
 // 12 warps = 3 warpgroups: two softmax warpgroups (warps 0-3, 4-7) and one
-// producer warpgroup (warp 8 issues the S MMAs, warp 9 the TMA loads, warp 10
-// the P V MMAs, warp 11 idles).  Launched at 168 registers per thread (the per-SM-sub-partition
+// producer warpgroup (warp 8 issues the S MMAs, warp 9 the TMA loads of Q and
+// K, warp 10 the P V MMAs, warp 11 the TMA loads of V).  Launched at 168 registers per thread (the per-SM-sub-partition
 // limit for 3 warps each); the producer warpgroup then gives registers up
 // and the softmax warpgroups take them: 2 * 128 * 200 + 128 * 96 = 63488 <=
 // 384 * 168, so the increase never waits on registers that do not exist.
 constexpr int NUM_THREADS = 384;
 constexpr int MMA_WARP = 8;    // issues S = Q K^T
-constexpr int LOAD_WARP = 9;
+constexpr int LOAD_WARP = 9;   // TMA loads of Q and K
 constexpr int PV_WARP = 10;    // issues O += P V
+constexpr int VLOAD_WARP = 11; // TMA loads of V
 constexpr uint32_t SOFTMAX_REGS = 200;
 constexpr uint32_t PRODUCER_REGS = 96;
 static_assert(2 * 128 * SOFTMAX_REGS + 128 * PRODUCER_REGS <= NUM_THREADS * 168,
@@ -99,7 +100,7 @@ struct SmemLayout {
   static constexpr int HALVES = D / 64;
   static constexpr int TILE_BYTES = HALVES * HALF_BYTES;
   // separate K and V rings, filled in the order the MMA warp consumes them
-  static constexpr int K_STAGES = (D == 64) ? 4 : 2;
+  static constexpr int K_STAGES = (D == 64) ? 4 : 3;
   static constexpr int V_STAGES = (D == 64) ? 4 : 2;
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
@@ -275,8 +276,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == LOAD_WARP && lane == 0) {
     prefetch_tensormap(&tm_q);
     prefetch_tensormap(&tm_k);
-    prefetch_tensormap(&tm_v);
   }
+  if (warp == VLOAD_WARP && lane == 0) prefetch_tensormap(&tm_v);
   if (warp == MMA_WARP) {
     tmem_alloc(smem_addr(tmem_slot), L::TMEM_COLS);
     tmem_relinquish();
@@ -301,84 +302,64 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool r = wait_phase(b, parity, abort_flag, site);
       return __all_sync(0xffffffffu, r);
     };
-    if (warp == LOAD_WARP) {
-      // ----------------------------------------------------------- TMA producer
-      // K_j and V_j are loaded in exactly the order the MMA warp first needs
-      // them (the same walk over the S sequence), each into its own ring.
-      uint32_t kpos = 0, vpos = 0, items_done = 0;
+    if (warp == LOAD_WARP || warp == VLOAD_WARP) {
+      // ----------------------------------------------------------- TMA producers
+      // Warp 9 loads each item's two Q tiles and K_0..K_{n-1}; warp 11 loads
+      // V_0..V_{n-1}.  Each ring is consumed in increasing j, so each loader
+      // streams its ring in that order and neither waits behind the other's
+      // free slots.
+      const bool is_k = (warp == LOAD_WARP);
+      const int stages = is_k ? L::K_STAGES : L::V_STAGES;
+      const uint32_t ring = is_k ? k_smem : v_smem;
+      const int full0 = is_k ? L::K_FULL : L::V_FULL;
+      const int empty0 = is_k ? L::K_EMPTY : L::V_EMPTY;
+      const CUtensorMap* map = is_k ? &tm_k : &tm_v;
+      uint32_t pos = 0, items_done = 0;
       bool ok = true;
       for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
         const int items = unit_items(p, u);
         for (int item = 0; ok && item < items; ++item) {
           const Unit w = decode_item(p, u, item);
-          if (items_done > 0) {
-            ok = warp_wait(bar(L::Q_EMPTY), (items_done - 1) & 1, SITE_LOAD_Q_EMPTY);
-            if (!ok) break;
-          }
-          if (leader) {
-            mbar_arrive_expect_tx(bar(L::Q_FULL), 2 * L::TILE_BYTES);
+          if (is_k) {
+            if (items_done > 0) {
+              ok = warp_wait(bar(L::Q_EMPTY), (items_done - 1) & 1, SITE_LOAD_Q_EMPTY);
+              if (!ok) break;
+            }
+            if (leader) {
+              mbar_arrive_expect_tx(bar(L::Q_FULL), 2 * L::TILE_BYTES);
 #pragma unroll
-            for (int t = 0; t < 2; ++t)
+              for (int t = 0; t < 2; ++t)
+#pragma unroll
+                for (int h = 0; h < L::HALVES; ++h)
+                  tma_load_3d(q_smem + t * L::TILE_BYTES + h * L::HALF_BYTES, &tm_q,
+                              bar(L::Q_FULL), h * 64, w.q0 + t * BLOCK_M, w.bh);
+            }
+            __syncwarp();
+          }
+          ++items_done;
+          for (int j = 0; ok && j < w.nmax; ++j) {
+            const uint32_t st = pos % stages, ph = (pos / stages) & 1;
+            if (pos >= static_cast<uint32_t>(stages) &&
+                !warp_wait(bar(empty0 + st), ph ^ 1, SITE_LOAD_KV_EMPTY)) {
+              ok = false;
+              break;
+            }
+            if (leader) {
+              mbar_arrive_expect_tx(bar(full0 + st), L::TILE_BYTES);
 #pragma unroll
               for (int h = 0; h < L::HALVES; ++h)
-                tma_load_3d(q_smem + t * L::TILE_BYTES + h * L::HALF_BYTES, &tm_q, bar(L::Q_FULL),
-                            h * 64, w.q0 + t * BLOCK_M, w.bh);
-          }
-          __syncwarp();
-          ++items_done;
-          int k_next = 0, v_next = 0;
-          auto load_k_upto = [&](int j) -> bool {
-            for (; k_next <= j; ++k_next) {
-              const uint32_t st = kpos % L::K_STAGES, ph = (kpos / L::K_STAGES) & 1;
-              if (kpos >= static_cast<uint32_t>(L::K_STAGES) &&
-                  !warp_wait(bar(L::K_EMPTY + st), ph ^ 1, SITE_LOAD_KV_EMPTY))
-                return false;
-              if (leader) {
-                mbar_arrive_expect_tx(bar(L::K_FULL + st), L::TILE_BYTES);
-#pragma unroll
-                for (int h = 0; h < L::HALVES; ++h)
-                  tma_load_3d(k_smem + st * L::TILE_BYTES + h * L::HALF_BYTES, &tm_k,
-                              bar(L::K_FULL + st), h * 64, k_next * BLOCK_N, w.bh);
-              }
-              __syncwarp();
-              ++kpos;
+                tma_load_3d(ring + st * L::TILE_BYTES + h * L::HALF_BYTES, map, bar(full0 + st),
+                            h * 64, j * BLOCK_N, w.bh);
             }
-            return true;
-          };
-          auto load_v_upto = [&](int j) -> bool {
-            for (; v_next <= j; ++v_next) {
-              const uint32_t st = vpos % L::V_STAGES, ph = (vpos / L::V_STAGES) & 1;
-              if (vpos >= static_cast<uint32_t>(L::V_STAGES) &&
-                  !warp_wait(bar(L::V_EMPTY + st), ph ^ 1, SITE_LOAD_KV_EMPTY))
-                return false;
-              if (leader) {
-                mbar_arrive_expect_tx(bar(L::V_FULL + st), L::TILE_BYTES);
-#pragma unroll
-                for (int h = 0; h < L::HALVES; ++h)
-                  tma_load_3d(v_smem + st * L::TILE_BYTES + h * L::HALF_BYTES, &tm_v,
-                              bar(L::V_FULL + st), h * 64, v_next * BLOCK_N, w.bh);
-              }
-              __syncwarp();
-              ++vpos;
-            }
-            return true;
-          };
-          const int total = w.n[0] + w.n[1];
-          for (int k = 0; ok && k < min(NSB, total); ++k) ok = load_k_upto(seq_at(w, k).j);
-          for (int k = 0; ok && k < total; ++k) {
-            ok = load_v_upto(seq_at(w, k).j);
-            if (ok && k + NSB < total) ok = load_k_upto(seq_at(w, k + NSB).j);
+            __syncwarp();
+            ++pos;
           }
         }
       }
       // Every issued load must have landed before the CTA may exit.
-      for (uint32_t i = kpos > L::K_STAGES ? kpos - L::K_STAGES : 0; i < kpos; ++i)
-        wait_phase(bar(L::K_FULL + i % L::K_STAGES), (i / L::K_STAGES) & 1, abort_flag, SITE_DRAIN,
-                   false);
-      for (uint32_t i = vpos > L::V_STAGES ? vpos - L::V_STAGES : 0; i < vpos; ++i)
-        wait_phase(bar(L::V_FULL + i % L::V_STAGES), (i / L::V_STAGES) & 1, abort_flag, SITE_DRAIN,
-                   false);
-      if (items_done > 0)
+      for (uint32_t i = pos > static_cast<uint32_t>(stages) ? pos - stages : 0; i < pos; ++i)
+        wait_phase(bar(full0 + i % stages), (i / stages) & 1, abort_flag, SITE_DRAIN, false);
+      if (is_k && items_done > 0)
         wait_phase(bar(L::Q_FULL), (items_done - 1) & 1, abort_flag, SITE_DRAIN, false);
       __syncwarp();
     } else if (warp == MMA_WARP || warp == PV_WARP) {
