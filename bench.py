@@ -291,10 +291,15 @@ def main():
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
     code = attn.ATTN_BF16 if w.dtype == "bf16" else attn.ATTN_FP16
     sh = stream.cuda_stream
+    # split-mode workspace (allocated once, outside the timed region; None when unused)
+    ws = attn.workspace_for(qd, kd, w.causal)
+    ws_ptr = ws.data_ptr() if ws is not None else None
+    ws_bytes = ws.numel() if ws is not None else 0
 
     def step():
-        st = attn.attn_fwd(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
-                           ld.data_ptr(), w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, code, sh)
+        st = attn.attn_fwd_ws(qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(),
+                              ld.data_ptr(), w.B, w.H, w.Nq, w.Nk, w.d, w.scale, w.causal, code,
+                              ws_ptr, ws_bytes, sh)
         if st != 0:
             raise attn.AttnError(st)
 
@@ -340,8 +345,8 @@ def main():
     def e2e_step():
         st = attn.attn_fwd_host(qh.data_ptr(), kh.data_ptr(), vh.data_ptr(), oh.data_ptr(),
                                 lh.data_ptr(), qd.data_ptr(), kd.data_ptr(), vd.data_ptr(),
-                                od.data_ptr(), ld.data_ptr(), w.B, w.H, w.Nq, w.Nk, w.d, w.scale,
-                                w.causal, code, sh)
+                                od.data_ptr(), ld.data_ptr(), ws_ptr, ws_bytes, w.B, w.H, w.Nq,
+                                w.Nk, w.d, w.scale, w.causal, code, sh)
         if st != 0:
             raise attn.AttnError(st, "attn_fwd_host")
 
@@ -396,6 +401,7 @@ def main():
                     "ms_per_step": round(e2e_ms / args.steps, 4),
                     "path": "attn_fwd_host: pinned host -> device, kernel, device -> host"},
             "gpu_launches": args.steps,
+            "split_mode": ws is not None,
             "clocks": sampler.summary(),
             "kernel_source_sha": kernel_source_sha(),
         }
@@ -416,20 +422,22 @@ def context_timings(attn, torch, dev, peaks, steps=10):
         q, k, v = (t.to(dev) for t in make_workload_qkv(w))
         o = torch.empty_like(q)
         lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+        ws = attn.workspace_for(q, k, w.causal)
         for _ in range(3):
-            attn.forward(q, k, v, causal=w.causal, out=o, lse=lse)
+            attn.forward(q, k, v, causal=w.causal, out=o, lse=lse, workspace=ws)
         times = []
         for _ in range(steps):
             flush.zero_()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            attn.forward(q, k, v, causal=w.causal, out=o, lse=lse)
+            attn.forward(q, k, v, causal=w.causal, out=o, lse=lse, workspace=ws)
             e1.record()
             torch.cuda.synchronize()
             times.append(e0.elapsed_time(e1))
         us = statistics.median(times) * 1e3
         r = roofline(w, us * 1e-6, peaks)
-        out[w.name] = {"us_per_call": round(us, 2), "tflops": round(w.flops / (us * 1e-6) / 1e12, 2),
+        out[w.name] = {"us_per_call": round(us, 2), "split": ws is not None,
+                       "tflops": round(w.flops / (us * 1e-6) / 1e12, 2),
                        "bound": r["bound"], "frac": r["frac"],
                        "frac_of_sustained": roofline(w, us * 1e-6, peaks, sustained=True)["frac"]}
         del q, k, v, o, lse

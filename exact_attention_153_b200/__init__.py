@@ -21,7 +21,7 @@ import os
 __all__ = [
     "ATTN_FP16", "ATTN_BF16", "AttnError", "lib", "library_path", "attn_fwd", "attn_fwd_host",
     "attn_plan", "attn_get_device_status", "attn_strerror", "attn_version", "forward",
-    "forward_host", "STATUS_NAMES",
+    "forward_host", "STATUS_NAMES", "attn_fwd_ws", "attn_workspace_size", "workspace_for",
 ]
 
 ATTN_FP16 = 0
@@ -55,7 +55,9 @@ class _Plan(ctypes.Structure):
                 ("num_kv_tiles", ctypes.c_int), ("units_per_head", ctypes.c_int),
                 ("num_units", ctypes.c_int),
                 ("grid", ctypes.c_int), ("block", ctypes.c_int), ("smem_bytes", ctypes.c_int),
-                ("stages", ctypes.c_int), ("qk_tile_products", ctypes.c_longlong)]
+                ("stages", ctypes.c_int), ("qk_tile_products", ctypes.c_longlong),
+                ("split", ctypes.c_int), ("split_grid", ctypes.c_int),
+                ("workspace_bytes", ctypes.c_longlong)]
 
 
 def lib() -> ctypes.CDLL:
@@ -71,7 +73,12 @@ def lib() -> ctypes.CDLL:
         vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
         L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
         L.attn_fwd.restype = i
-        L.attn_fwd_host.argtypes = [vp] * 10 + [i, i, i, i, i, f, i, i, vp]
+        L.attn_fwd_ws.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, ctypes.c_size_t,
+                                  vp]
+        L.attn_fwd_ws.restype = i
+        L.attn_workspace_size.argtypes = [i, i, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
+        L.attn_workspace_size.restype = i
+        L.attn_fwd_host.argtypes = [vp] * 11 + [ctypes.c_size_t, i, i, i, i, i, f, i, i, vp]
         L.attn_fwd_host.restype = i
         L.attn_plan.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(_Plan)]
         L.attn_plan.restype = i
@@ -92,11 +99,28 @@ def attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, stream) -> 
     return lib().attn_fwd(q, k, v, o, lse, B, H, Nq, Nk, d, float(scale), int(causal), dtype, stream)
 
 
-def attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, B, H, Nq, Nk, d, scale,
-                  causal, dtype, stream) -> int:
+def attn_fwd_ws(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, workspace, ws_bytes,
+                stream) -> int:
+    """Raw ``attn_fwd_ws``: attn_fwd with a device workspace (split mode)."""
+    return lib().attn_fwd_ws(q, k, v, o, lse, B, H, Nq, Nk, d, float(scale), int(causal), dtype,
+                             workspace, ws_bytes, stream)
+
+
+def attn_workspace_size(B, H, Nq, Nk, d, causal) -> int:
+    """Workspace bytes attn_fwd_ws uses for these sizes on the current device."""
+    n = ctypes.c_size_t(0)
+    st = lib().attn_workspace_size(B, H, Nq, Nk, d, int(causal), ctypes.byref(n))
+    if st != 0:
+        raise AttnError(st, "attn_workspace_size")
+    return n.value
+
+
+def attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, workspace, ws_bytes, B,
+                  H, Nq, Nk, d, scale, causal, dtype, stream) -> int:
     """Raw ``attn_fwd_host``: host and device pointers as Python ints."""
-    return lib().attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, B, H, Nq,
-                               Nk, d, float(scale), int(causal), dtype, stream)
+    return lib().attn_fwd_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, workspace,
+                               ws_bytes, B, H, Nq, Nk, d, float(scale), int(causal), dtype,
+                               stream)
 
 
 def attn_plan(B, H, Nq, Nk, d, causal, num_sms) -> dict:
@@ -144,7 +168,7 @@ def _dtype_code(t) -> int:
 
 
 def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None, lse=None,
-            return_lse: bool = True, stream=None):
+            return_lse: bool = True, stream=None, workspace=None):
     """Attention forward on CUDA tensors [B, H, N, d]; returns (o, lse).
 
     ``scale`` defaults to 1/sqrt(d), the default of the pages' SDPA call
@@ -172,16 +196,32 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
         out = torch.empty((B, H, Nq, d), dtype=q.dtype, device=q.device)
     if lse is None and return_lse:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
-    st = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
-                  lse.data_ptr() if lse is not None else None, B, H, Nq, Nk, d, scale, causal,
-                  code, _stream_handle(stream))
+    if workspace is None:
+        st = attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                      lse.data_ptr() if lse is not None else None, B, H, Nq, Nk, d, scale, causal,
+                      code, _stream_handle(stream))
+    else:
+        st = attn_fwd_ws(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                         lse.data_ptr() if lse is not None else None, B, H, Nq, Nk, d, scale,
+                         causal, code, workspace.data_ptr(),
+                         workspace.numel() * workspace.element_size(), _stream_handle(stream))
     if st != 0:
         raise AttnError(st)
     return out, lse
 
 
+def workspace_for(q, k, causal: bool = False):
+    """A zero-filled device workspace sized for attn_fwd_ws on these inputs (or None)."""
+    import torch
+    B, H, Nq, d = q.shape
+    n = attn_workspace_size(B, H, Nq, k.shape[2], d, causal)
+    if n == 0:
+        return None
+    return torch.zeros(n, dtype=torch.uint8, device=q.device)
+
+
 def forward_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal=False, scale=None,
-                 stream=None):
+                 stream=None, workspace=None):
     """End-to-end call from (pinned) host tensors through caller-owned device buffers."""
     B, H, Nq, d = q_h.shape
     Nk = k_h.shape[2]
@@ -191,6 +231,8 @@ def forward_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal=Fa
                        lse_h.data_ptr() if lse_h is not None else None,
                        q_d.data_ptr(), k_d.data_ptr(), v_d.data_ptr(), o_d.data_ptr(),
                        lse_d.data_ptr() if lse_d is not None else None,
+                       workspace.data_ptr() if workspace is not None else None,
+                       workspace.numel() * workspace.element_size() if workspace is not None else 0,
                        B, H, Nq, Nk, d, scale, causal, _dtype_code(q_h), _stream_handle(stream))
     if st != 0:
         raise AttnError(st, "attn_fwd_host")

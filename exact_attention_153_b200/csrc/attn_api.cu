@@ -50,7 +50,7 @@ struct DeviceInfo {
   bool probed = false;
   bool supported = false;
   int sms = 0;
-  bool smem_attr[2][2] = {{false, false}, {false, false}};  // [d==128][bf16]
+  bool smem_attr[2][2][2] = {};  // [d==128][bf16][split]
 };
 
 std::mutex g_dev_mutex;
@@ -81,6 +81,23 @@ int check_args(const void* q, const void* k, const void* v, const void* o, const
   return ATTN_OK;
 }
 
+// Split mode pays off when whole units would leave a ragged last wave: the
+// CTAs that run one unit more set the kernel time.  It needs a workspace and
+// is used for non-causal problems whose unit count spreads over the grid
+// with less than 90 % efficiency.
+bool split_pays(long long units, long long total_steps, int num_sms, int causal) {
+  if (causal || total_steps < 2) return false;
+  const long long grid = units < num_sms ? units : num_sms;
+  const long long waves = (units + grid - 1) / grid;
+  const double eff = static_cast<double>(units) / static_cast<double>(grid * waves);
+  return eff < 0.9 || units < num_sms;
+}
+
+size_t split_workspace_bytes(int grid, int d, long long units) {
+  const size_t rows = static_cast<size_t>(grid) * 2 * 2 * BLOCK_M;
+  return rows * d * sizeof(float) + rows * sizeof(float) + static_cast<size_t>(units) * 4 + 16;
+}
+
 void fill_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, attn_plan_t* out) {
   const int q_tiles = ceil_div(Nq, BLOCK_M);
   const int q_pairs = ceil_div(q_tiles, 2);
@@ -109,6 +126,11 @@ void fill_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, att
     }
   }
   out->qk_tile_products = per_head * B * H;
+  const long long total_steps = units * kv_tiles;
+  out->split = split_pays(units, total_steps, num_sms, causal) ? 1 : 0;
+  out->split_grid = static_cast<int>(total_steps < num_sms ? total_steps : num_sms);
+  out->workspace_bytes =
+      out->split ? static_cast<long long>(split_workspace_bytes(out->split_grid, d, units)) : 0;
 }
 
 // Probe the current device once: compute capability 10.0 and SM count.
@@ -171,12 +193,12 @@ struct MapCache {
 };
 thread_local MapCache t_maps;
 
-template <int D, bool BF16>
-int launch(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo& info,
-           cudaStream_t stream) {
-  auto kernel = attn_sm100::attn_fwd_kernel<D, BF16>;
+template <int D, bool BF16, bool SPLIT>
+int launch_one(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo& info,
+               cudaStream_t stream) {
+  auto kernel = attn_sm100::attn_fwd_kernel<D, BF16, SPLIT>;
   constexpr int smem = SmemLayout<D>::BYTES;
-  bool& attr = info.smem_attr[D == 128][BF16];
+  bool& attr = info.smem_attr[D == 128][BF16][SPLIT];
   if (!attr) {
     std::lock_guard<std::mutex> lock(g_dev_mutex);
     if (!attr) {
@@ -192,12 +214,18 @@ int launch(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo& inf
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-}  // namespace
+// Split mode is a separate instantiation, so the unit-mode kernel carries none
+// of the piece bookkeeping.
+template <int D, bool BF16>
+int launch(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo& info,
+           cudaStream_t stream) {
+  return prm.split ? launch_one<D, BF16, true>(maps, prm, grid, info, stream)
+                   : launch_one<D, BF16, false>(maps, prm, grid, info, stream);
+}
 
-extern "C" {
-
-int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-             int Nq, int Nk, int d, float scale, int causal, int dtype, attn_stream_t stream) {
+static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int H, int Nq, int Nk, int d, float scale, int causal, int dtype,
+                    void* workspace, size_t workspace_bytes, attn_stream_t stream) {
   int st = check_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, dtype);
   if (st != ATTN_OK) return st;
   int dev = -1;
@@ -232,19 +260,69 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   prm.num_units = plan.num_units;
   prm.causal = causal ? 1 : 0;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  prm.split = 0;
+  prm.total_steps = 0;
+  prm.ws_o = nullptr;
+  prm.ws_lse = nullptr;
+  prm.ws_count = nullptr;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int grid = plan.grid;
+  if (plan.split && workspace != nullptr &&
+      workspace_bytes >= static_cast<size_t>(plan.workspace_bytes) &&
+      (reinterpret_cast<uintptr_t>(workspace) & 15) == 0) {
+    grid = plan.split_grid;
+    const size_t rows = static_cast<size_t>(grid) * 2 * 2 * BLOCK_M;
+    char* ws = static_cast<char*>(workspace);
+    prm.split = 1;
+    prm.total_steps = static_cast<long long>(plan.num_units) * plan.num_kv_tiles;
+    prm.ws_o = reinterpret_cast<float*>(ws);
+    prm.ws_lse = reinterpret_cast<float*>(ws + rows * d * sizeof(float));
+    // the piece counters start at zero (the caller zero-fills a new
+    // workspace) and every completed call leaves them at zero again
+    prm.ws_count = reinterpret_cast<unsigned int*>(ws + rows * (d + 1) * sizeof(float));
+  }
   if (d == 64)
-    return dtype == ATTN_BF16 ? launch<64, true>(mc, prm, plan.grid, *info, s)
-                              : launch<64, false>(mc, prm, plan.grid, *info, s);
-  return dtype == ATTN_BF16 ? launch<128, true>(mc, prm, plan.grid, *info, s)
-                            : launch<128, false>(mc, prm, plan.grid, *info, s);
+    return dtype == ATTN_BF16 ? launch<64, true>(mc, prm, grid, *info, s)
+                              : launch<64, false>(mc, prm, grid, *info, s);
+  return dtype == ATTN_BF16 ? launch<128, true>(mc, prm, grid, *info, s)
+                            : launch<128, false>(mc, prm, grid, *info, s);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+             int Nq, int Nk, int d, float scale, int causal, int dtype, attn_stream_t stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, nullptr, 0, stream);
+}
+
+int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                int Nq, int Nk, int d, float scale, int causal, int dtype, void* workspace,
+                size_t workspace_bytes, attn_stream_t stream) {
+  return fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, workspace,
+                  workspace_bytes, stream);
+}
+
+int attn_workspace_size(int B, int H, int Nq, int Nk, int d, int causal, size_t* bytes) {
+  if (bytes == nullptr) return ATTN_ERR_NULL;
+  if (d != 64 && d != 128) return ATTN_ERR_HEAD_DIM;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return ATTN_ERR_SHAPE;
+  int dev = -1;
+  DeviceInfo* info = nullptr;
+  const int st = current_device(&dev, &info);
+  if (st != ATTN_OK) return st;
+  attn_plan_t plan;
+  fill_plan(B, H, Nq, Nk, d, causal, info->sms, &plan);
+  *bytes = static_cast<size_t>(plan.workspace_bytes);
+  return ATTN_OK;
 }
 
 int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
                   float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
-                  float* lse_dev, int B, int H, int Nq, int Nk, int d, float scale, int causal,
-                  int dtype, attn_stream_t stream) {
+                  float* lse_dev, void* workspace, size_t workspace_bytes, int B, int H, int Nq,
+                  int Nk, int d, float scale, int causal, int dtype, attn_stream_t stream) {
   if (q_host == nullptr || k_host == nullptr || v_host == nullptr || o_host == nullptr)
     return ATTN_ERR_NULL;
   int st = check_args(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Nq, Nk, d, scale, dtype);
@@ -258,7 +336,8 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }
-  st = attn_fwd(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Nq, Nk, d, scale, causal, dtype, stream);
+  st = fwd_impl(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Nq, Nk, d, scale, causal, dtype,
+                workspace, workspace_bytes, stream);
   if (st != ATTN_OK) return st;
   if (cudaMemcpyAsync(o_host, o_dev, q_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
       (lse_host != nullptr && lse_dev != nullptr &&

@@ -48,16 +48,23 @@ constexpr int BLOCK_N = 128;     // keys per K / V tile
 // producer warpgroup (warp 8 issues the S MMAs, warp 9 the TMA loads of Q and
 // K, warp 10 the P V MMAs, warp 11 the TMA loads of V).  Launched at 168 registers per thread (the per-SM-sub-partition
 // limit for 3 warps each); the producer warpgroup then gives registers up
-// and the softmax warpgroups take them: 2 * 128 * 200 + 128 * 96 = 63488 <=
-// 384 * 168, so the increase never waits on registers that do not exist.
+// and the softmax warpgroups take them (2 * 128 * 200 + 128 * 96 = 63488, or
+// 2 * 128 * 208 + 128 * 88 = 64512, both <= 384 * 168), so the increase never
+// waits on registers that do not exist.
 constexpr int NUM_THREADS = 384;
 constexpr int MMA_WARP = 8;    // issues S = Q K^T
 constexpr int LOAD_WARP = 9;   // TMA loads of Q and K
 constexpr int PV_WARP = 10;    // issues O += P V
 constexpr int VLOAD_WARP = 11; // TMA loads of V
-constexpr uint32_t SOFTMAX_REGS = 200;
-constexpr uint32_t PRODUCER_REGS = 96;
-static_assert(2 * 128 * SOFTMAX_REGS + 128 * PRODUCER_REGS <= NUM_THREADS * 168,
+// The split-mode kernel (piece bookkeeping and merge in the softmax) needs a
+// few more softmax registers than the unit-mode one.
+template <bool SPLIT>
+__host__ __device__ constexpr uint32_t softmax_regs() { return SPLIT ? 208 : 200; }
+template <bool SPLIT>
+__host__ __device__ constexpr uint32_t producer_regs() { return SPLIT ? 88 : 96; }
+static_assert(2 * 128 * softmax_regs<true>() + 128 * producer_regs<true>() <= NUM_THREADS * 168,
+              "register split exceeds the launch budget");
+static_assert(2 * 128 * softmax_regs<false>() + 128 * producer_regs<false>() <= NUM_THREADS * 168,
               "register split exceeds the launch budget");
 constexpr uint64_t WAIT_LIMIT_NS = 1000000000ull;
 constexpr float RESCALE_LOG2 = 8.0f;  // lazy-rescale threshold for the running max
@@ -92,6 +99,17 @@ struct FwdParams {
   int num_units;    // BH * units_per_head
   int causal;
   float scale_log2; // scale * log2(e)
+  // Split mode (non-causal only).  The units' key tiles are flattened into
+  // total_steps = num_units * num_kv_tiles steps and CTA c takes steps
+  // [c * total_steps / grid, (c + 1) * total_steps / grid), so every CTA does
+  // the same work however the units divide.  A unit cut by a range boundary
+  // is computed in pieces; each piece leaves its normalised O and lse in the
+  // caller's workspace and the last piece to finish merges them.
+  int split;
+  long long total_steps;
+  float* ws_o;           // [grid][2 slots][2 tiles][128 rows][D]
+  float* ws_lse;         // [grid][2 slots][2 tiles][128 rows]
+  unsigned int* ws_count;  // [num_units] pieces finished; zero between calls
 };
 
 template <int D>
@@ -137,9 +155,11 @@ struct SmemLayout {
 
 struct Unit {
   int bh;
-  int q0;    // first query row of tile 0
-  int n[2];  // K/V tiles each Q tile visits (0 = tile lies past Nq)
+  int q0;     // first query row of tile 0
+  int jbase;  // first K/V tile of this item (non-zero only for split pieces)
+  int n[2];   // K/V tiles each Q tile visits from jbase (0 = tile lies past Nq)
   int nmax;
+  int unit, piece, pieces, c_first;  // split pieces: which, how many, CTA of piece 0
 };
 
 // Work schedule.  A work unit belongs to one (batch, head) and holds one or
@@ -183,7 +203,85 @@ __device__ __forceinline__ Unit decode_item(const FwdParams& p, int u, int item)
     w.n[t] = n;
   }
   w.nmax = max(w.n[0], w.n[1]);
+  w.jbase = 0;
+  w.unit = u;
+  w.piece = 0;
+  w.pieces = 1;
+  w.c_first = 0;
   return w;
+}
+
+// Iterates the items of this CTA, identically in every role.
+template <bool SPLIT>
+struct WorkCursor {
+  int u, item, items;
+  long long idx, end;
+  __device__ __forceinline__ explicit WorkCursor(const FwdParams& p) {
+    if constexpr (SPLIT) {
+      idx = p.total_steps * blockIdx.x / gridDim.x;
+      end = p.total_steps * (blockIdx.x + 1) / gridDim.x;
+      u = item = items = 0;
+    } else {
+      u = blockIdx.x;
+      item = 0;
+      items = u < p.num_units ? unit_items(p, u) : 0;
+      idx = end = 0;
+    }
+  }
+  // Number of CTAs c >= 1 whose step range begins at or before step x.
+  __device__ __forceinline__ static long long starts_le(const FwdParams& p, long long x) {
+    const long long g = gridDim.x;
+    const long long c = ((x + 1) * g - 1) / p.total_steps;
+    return c < g - 1 ? c : g - 1;
+  }
+  __device__ __forceinline__ bool next(const FwdParams& p, Unit& w) {
+    if constexpr (SPLIT) {
+      if (idx >= end) return false;
+      const int nk = p.num_kv_tiles;
+      const int uu = static_cast<int>(idx / nk);
+      const int j0 = static_cast<int>(idx % nk);
+      const long long left = end - idx;
+      const int j1 = left < nk - j0 ? j0 + static_cast<int>(left) : nk;
+      w = decode_item(p, uu, 0);
+      w.jbase = j0;
+      w.n[0] = w.n[0] > 0 ? j1 - j0 : 0;
+      w.n[1] = w.n[1] > 0 ? j1 - j0 : 0;
+      w.nmax = max(w.n[0], w.n[1]);
+      const long long a = static_cast<long long>(uu) * nk;
+      const long long ca = starts_le(p, a);
+      w.piece = static_cast<int>(starts_le(p, a + j0) - ca);
+      w.pieces = static_cast<int>(1 + starts_le(p, a + nk - 1) - ca);
+      w.c_first = static_cast<int>(ca);
+      idx += j1 - j0;
+      return true;
+    } else {
+      while (item >= items) {
+        u += gridDim.x;
+        if (u >= p.num_units) return false;
+        item = 0;
+        items = unit_items(p, u);
+      }
+      w = decode_item(p, u, item++);
+      return true;
+    }
+  }
+};
+
+// Piece k of a split unit lives in CTA (c_first + k): piece 0 is that CTA's
+// last item (it runs to the end of the CTA's range), every later piece is
+// its CTA's first item (it starts the range), so one CTA holds at most one
+// piece in each of its two workspace slots.
+__device__ __forceinline__ size_t ws_row(int cta, int slot, int t, int r) {
+  return ((static_cast<size_t>(cta) * 2 + slot) * 2 + t) * BLOCK_M + r;
+}
+// A slot's O is stored column-major (column c of row r at c * 128 + r), so
+// the 32 rows of a warp read and write 32 consecutive floats.
+__device__ __forceinline__ size_t ws_o_base(int cta, int slot, int t, int D) {
+  return ((static_cast<size_t>(cta) * 2 + slot) * 2 + t) * static_cast<size_t>(BLOCK_M) * D;
+}
+
+__device__ __forceinline__ void softmax_barrier() {
+  asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight softmax warps only
 }
 
 // The S sequence of one item: the MMA warp computes the score tiles of the
@@ -233,7 +331,7 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
   return true;
 }
 
-template <int D, bool BF16>
+template <int D, bool BF16, bool SPLIT>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -288,7 +386,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const uint32_t tmem_base = *tmem_slot;
 
   if (warp >= 8) {
-    regs_decrease<PRODUCER_REGS>();
+    regs_decrease<producer_regs<SPLIT>()>();
     // The producer warps run their loops on all 32 lanes, so every address,
     // coordinate and descriptor is warp-uniform and stays in uniform
     // registers; one elected lane issues the TMA and tcgen05 instructions
@@ -316,10 +414,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const CUtensorMap* map = is_k ? &tm_k : &tm_v;
       uint32_t pos = 0, items_done = 0;
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-        const int items = unit_items(p, u);
-        for (int item = 0; ok && item < items; ++item) {
-          const Unit w = decode_item(p, u, item);
+      WorkCursor<SPLIT> cur(p);
+      Unit w;
+      while (ok && cur.next(p, w)) {
+        {
           if (is_k) {
             if (items_done > 0) {
               ok = warp_wait(bar(L::Q_EMPTY), (items_done - 1) & 1, SITE_LOAD_Q_EMPTY);
@@ -349,7 +447,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int h = 0; h < L::HALVES; ++h)
                 tma_load_3d(ring + st * L::TILE_BYTES + h * L::HALF_BYTES, map, bar(full0 + st),
-                            h * 64, j * BLOCK_N, w.bh);
+                            h * 64, (w.jbase + j) * BLOCK_N, w.bh);
             }
             __syncwarp();
             ++pos;
@@ -401,10 +499,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t pos = 0, g = 0, q_phase = 0;  // ring position of K_0 / V_0 of the item; score tile count
       uint32_t buf = 0, round = 0;           // g % NSB, g / NSB
       bool ok = true;
-      for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-        const int items = unit_items(p, u);
-        for (int item = 0; ok && item < items; ++item) {
-          const Unit w = decode_item(p, u, item);
+      WorkCursor<SPLIT> cur(p);
+      Unit w;
+      while (ok && cur.next(p, w)) {
+        {
           const int total = w.n[0] + w.n[1];
           if (is_s) {
             ok = warp_wait(bar(L::Q_FULL), q_phase, SITE_MMA_Q_FULL);
@@ -553,7 +651,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
     }
   } else {
-    regs_increase<SOFTMAX_REGS>();
+    regs_increase<softmax_regs<SPLIT>()>();
     // ------------------------------------------------------------- softmax
     const int t = warp / 4;
     const int quarter = warp % 4;
@@ -565,14 +663,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t o_phase = 0, sk = 0;
     uint32_t s_parity = 0;  // bit b: parity of the next S_FULL(b, t) phase this warpgroup waits for
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < p.num_units; u += gridDim.x) {
-      const int items = unit_items(p, u);
-      for (int item = 0; ok && item < items; ++item) {
-        const Unit w = decode_item(p, u, item);
+    volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
+    WorkCursor<SPLIT> cur(p);
+    Unit w;
+    while (ok && cur.next(p, w)) {
+      {
         const int n = t ? w.n[1] : w.n[0];
         const uint32_t item_sk = sk;
         sk += w.n[0] + w.n[1];
-        if (n == 0) continue;
+        if (n == 0 && (!SPLIT || w.pieces == 1)) continue;
         const int q_start = w.q0 + t * BLOCK_M;
         const int row = q_start + r;
         // last key this row may see (top-left causal: key j <= query i)
@@ -597,7 +696,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
           for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
 
-          const int k0 = j * BLOCK_N;
+          const int k0 = (w.jbase + j) * BLOCK_N;
           const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > q_start);
           if (need_mask) {
             const int lim = last_key - k0;  // columns > lim are masked
@@ -688,33 +787,151 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (!ok) break;
 
         // --------------------------------------------------------- epilogue
-        ok = wait_phase(bar(L::O_READY + t), o_phase, abort_flag, SITE_SOFTMAX_O_READY);
-        ok = __all_sync(0xffffffffu, ok);
-        if (!ok) break;
-        o_phase ^= 1;
-        tc_fence_after();
-        const float inv_l = 1.f / l;
         const bool in_range = row < p.Nq;
-        uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
-                                               (static_cast<size_t>(w.bh) * p.Nq + row) * D);
+        float lse_self = 0.f, inv_self = 0.f;  // this piece's statistics, for the merge
+        if (n > 0) {
+          ok = wait_phase(bar(L::O_READY + t), o_phase, abort_flag, SITE_SOFTMAX_O_READY);
+          ok = __all_sync(0xffffffffu, ok);
+          if (!ok) break;
+          o_phase ^= 1;
+          tc_fence_after();
+          const float inv_l = 1.f / l;
+          const float lse_row = (m + lg2_approx(l)) * 0.69314718055994531f;
+          lse_self = lse_row;
+          inv_self = inv_l;
+          if (!SPLIT || w.pieces == 1) {
+            uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
+                                                   (static_cast<size_t>(w.bh) * p.Nq + row) * D);
 #pragma unroll
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          uint32_t o[32];
-          tmem_ld32(tO + c0, o);
-          tmem_wait_ld_regs(o);
-          uint32_t pk[16];
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32(tO + c0, o);
+              tmem_wait_ld_regs(o);
+              uint32_t pk[16];
 #pragma unroll
-          for (int i = 0; i < 16; ++i)
-            pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l, __uint_as_float(o[2 * i + 1]) * inv_l);
-          if (in_range) {
+              for (int i = 0; i < 16; ++i)
+                pk[i] = pack2<BF16>(__uint_as_float(o[2 * i]) * inv_l,
+                                    __uint_as_float(o[2 * i + 1]) * inv_l);
+              if (in_range) {
 #pragma unroll
-            for (int v4 = 0; v4 < 4; ++v4)
-              orow[c0 / 8 + v4] = make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+                for (int v4 = 0; v4 < 4; ++v4)
+                  orow[c0 / 8 + v4] =
+                      make_uint4(pk[4 * v4], pk[4 * v4 + 1], pk[4 * v4 + 2], pk[4 * v4 + 3]);
+              }
+            }
+            if (p.lse != nullptr && in_range)
+              p.lse[static_cast<size_t>(w.bh) * p.Nq + row] = lse_row;
+          } else {
+            // a piece of a split unit: normalised O and lse to this CTA's slot
+            const int slot = w.piece == 0 ? 1 : 0;
+            const size_t wr = ws_row(blockIdx.x, slot, t, r);
+            float* so = p.ws_o + ws_o_base(blockIdx.x, slot, t, D) + r;
+#pragma unroll
+            for (int c0 = 0; c0 < D; c0 += 32) {
+              uint32_t o[32];
+              tmem_ld32(tO + c0, o);
+              tmem_wait_ld_regs(o);
+              if (in_range) {
+#pragma unroll
+                for (int c = 0; c < 32; ++c)
+                  __stcg(so + static_cast<size_t>(c0 + c) * BLOCK_M, __uint_as_float(o[c]) * inv_l);
+              }
+            }
+            if (in_range) __stcg(p.ws_lse + wr, lse_row);
+          }
+          tc_fence_before();
+        }
+        if (SPLIT && w.pieces > 1) {
+          // Both warpgroups publish their rows, then one thread counts the
+          // piece; the CTA that brings the count to `pieces` merges all of
+          // them with the log-domain identity lse = ln sum_k e^{lse_k},
+          // O = sum_k e^{lse_k - lse} O_k, and resets the counter for the
+          // next call.
+          __threadfence();
+          softmax_barrier();
+          if (threadIdx.x == 0) {
+            const unsigned int done = atomicAdd(p.ws_count + w.unit, 1u);
+            const int last = (done == static_cast<unsigned int>(w.pieces - 1)) ? 1 : 0;
+            if (last) p.ws_count[w.unit] = 0u;
+            *last_flag = last;
+          }
+          softmax_barrier();
+          const bool last = *last_flag != 0;
+          softmax_barrier();  // everyone has read the flag before it is reused
+          const int n_unit = t ? (w.q0 + BLOCK_M < p.Nq) : 1;  // does tile t have rows at all
+          if (last && n_unit) {
+            // This CTA finished the unit's last piece.  Its own piece is still
+            // in TMEM; the others are read from their slots (coalesced: one
+            // column of 32 rows per warp load), all loads of a piece issued
+            // before any is used.
+            __threadfence();
+            tc_fence_after();
+            float lse_max = lse_self;
+            for (int k = 0; k < w.pieces; ++k) {
+              if (k == w.piece || !in_range) continue;
+              lse_max = fmaxf(lse_max, __ldcg(p.ws_lse + ws_row(w.c_first + k, k == 0 ? 1 : 0, t, r)));
+            }
+            const float w_self = ex2_approx((lse_self - lse_max) * 1.4426950408889634f);
+            float wsum = 0.f;
+            uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
+                                                   (static_cast<size_t>(w.bh) * p.Nq + row) * D);
+            // Pieces are summed in piece order whichever CTA merges, and the
+            // own piece's values are formed exactly as they were stored, so
+            // the result is bit-for-bit the same on every call.
+#pragma unroll 1
+            for (int h = 0; h < D / 64; ++h) {
+              float acc[64];
+#pragma unroll
+              for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+              float hsum = 0.f;
+              for (int k = 0; k < w.pieces; ++k) {
+                float wk;
+                float v[64];
+                if (k == w.piece) {
+                  wk = w_self;
+                  uint32_t o[32];
+#pragma unroll
+                  for (int c0 = 0; c0 < 64; c0 += 32) {
+                    tmem_ld32(tO + 64 * h + c0, o);
+                    tmem_wait_ld_regs(o);
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) v[c0 + c] = __uint_as_float(o[c]) * inv_self;
+                  }
+                } else {
+                  const int slot = k == 0 ? 1 : 0;
+                  wk = 0.f;
+#pragma unroll
+                  for (int c = 0; c < 64; ++c) v[c] = 0.f;
+                  if (in_range) {
+                    wk = ex2_approx((__ldcg(p.ws_lse + ws_row(w.c_first + k, slot, t, r)) - lse_max) *
+                                    1.4426950408889634f);
+                    const float* src = p.ws_o + ws_o_base(w.c_first + k, slot, t, D) +
+                                       static_cast<size_t>(64 * h) * BLOCK_M + r;
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) v[c] = __ldcg(src + static_cast<size_t>(c) * BLOCK_M);
+                  }
+                }
+                hsum += wk;
+#pragma unroll
+                for (int c = 0; c < 64; ++c) acc[c] = fmaf(wk, v[c], acc[c]);
+              }
+              wsum = hsum;
+              const float inv = 1.f / hsum;
+              if (in_range) {
+#pragma unroll
+                for (int c8 = 0; c8 < 8; ++c8)
+                  orow[8 * h + c8] =
+                      make_uint4(pack2<BF16>(acc[8 * c8] * inv, acc[8 * c8 + 1] * inv),
+                                 pack2<BF16>(acc[8 * c8 + 2] * inv, acc[8 * c8 + 3] * inv),
+                                 pack2<BF16>(acc[8 * c8 + 4] * inv, acc[8 * c8 + 5] * inv),
+                                 pack2<BF16>(acc[8 * c8 + 6] * inv, acc[8 * c8 + 7] * inv));
+              }
+            }
+            if (p.lse != nullptr && in_range)
+              p.lse[static_cast<size_t>(w.bh) * p.Nq + row] =
+                  lse_max + lg2_approx(wsum) * 0.69314718055994531f;
           }
         }
-        if (p.lse != nullptr && in_range)
-          p.lse[static_cast<size_t>(w.bh) * p.Nq + row] = (m + lg2_approx(l)) * 0.69314718055994531f;
-        tc_fence_before();
       }
     }
   }

@@ -28,6 +28,8 @@
 #ifndef ATTN_SM100_ATTN_H_
 #define ATTN_SM100_ATTN_H_
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -66,6 +68,9 @@ typedef struct {
   int smem_bytes;    /* dynamic shared memory per CTA                                     */
   int stages;        /* K/V shared-memory ring slots                                      */
   long long qk_tile_products; /* 128x128 score tiles computed (incl. masked tail tiles)   */
+  int split;         /* 1 if attn_fwd_ws would use split mode for these sizes (see below)  */
+  int split_grid;    /* CTAs launched in split mode: min(SM count, units * num_kv_tiles)   */
+  long long workspace_bytes; /* workspace attn_fwd_ws needs for split mode; 0 if unused    */
 } attn_plan_t;
 
 /*
@@ -94,6 +99,40 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
              int Nq, int Nk, int d, float scale, int causal, int dtype, attn_stream_t stream);
 
 /*
+ * attn_fwd_ws -- attn_fwd with a caller-provided device workspace that enables split mode.
+ *
+ * For non-causal problems whose work units would fill the GPU unevenly (a ragged last wave,
+ * or fewer units than SMs -- e.g. the 20x20 and 40x40 YOLO workloads), the kernel divides
+ * the flattened (unit, key tile) range evenly over the CTAs.  A unit cut by a range boundary
+ * is computed in pieces; each piece writes its normalised O and its logsumexp to the
+ * workspace and the last piece to finish merges them exactly with the log-domain identity
+ * lse = ln sum_k exp(lse_k), O = sum_k exp(lse_k - lse) O_k (the saved-statistics
+ * combination of the "log 域" accumulation, coreui.cn section "原理").  Results equal those
+ * of attn_fwd up to rounding.
+ *
+ *   workspace        device pointer, 16-byte aligned, at least attn_workspace_size() bytes,
+ *                    caller-owned.  Zero-fill it once before its first use (cudaMemset): it
+ *                    holds per-unit piece counters, and every completed call leaves them at
+ *                    zero again, so later calls need no clearing.  After a call that ends in
+ *                    ATTN_ERR_DEVICE_TIMEOUT the counters may be left non-zero: zero-fill
+ *                    the workspace again.  Calls that share a workspace must be ordered
+ *                    (same stream); calls that overlap on the GPU with one workspace race.
+ *   workspace_bytes  its size.  If the workspace is NULL, too small or misaligned, or split
+ *                    mode does not pay for these sizes, the call behaves exactly as attn_fwd.
+ * Other arguments, errors and asynchrony as attn_fwd.
+ */
+int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                int Nq, int Nk, int d, float scale, int causal, int dtype, void* workspace,
+                size_t workspace_bytes, attn_stream_t stream);
+
+/*
+ * attn_workspace_size -- bytes of workspace attn_fwd_ws uses for these sizes on the current
+ * device (0 when split mode is not used).  Errors: ATTN_ERR_NULL (bytes NULL),
+ * ATTN_ERR_HEAD_DIM, ATTN_ERR_SHAPE, ATTN_ERR_CUDA / ATTN_ERR_ARCH (no usable device).
+ */
+int attn_workspace_size(int B, int H, int Nq, int Nk, int d, int causal, size_t* bytes);
+
+/*
  * attn_fwd_host -- the same forward, end to end from host memory.
  *
  * Enqueues on `stream`: host->device copies of q_host, k_host, v_host into the caller's
@@ -102,12 +141,13 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
  * lse_host.  Host buffers should be pinned (cudaHostAlloc / cudaHostRegister) for the copies
  * to be asynchronous.  The caller synchronises `stream` before reading o_host.  Argument
  * rules and error codes are those of attn_fwd; every host and device pointer except the lse
- * pair must be non-NULL.  Nothing is allocated.
+ * pair must be non-NULL.  workspace / workspace_bytes are optional (NULL, 0) and act as in
+ * attn_fwd_ws.  Nothing is allocated.
  */
 int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
                   float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
-                  float* lse_dev, int B, int H, int Nq, int Nk, int d, float scale, int causal,
-                  int dtype, attn_stream_t stream);
+                  float* lse_dev, void* workspace, size_t workspace_bytes, int B, int H, int Nq,
+                  int Nk, int d, float scale, int causal, int dtype, attn_stream_t stream);
 
 /*
  * attn_plan -- the launch geometry attn_fwd would use for these sizes on a GPU with

@@ -33,8 +33,8 @@ def header_functions():
 
 def test_header_declares_the_boundary():
     assert header_functions() == sorted([
-        "attn_fwd", "attn_fwd_host", "attn_plan", "attn_get_device_status", "attn_strerror",
-        "attn_version"])
+        "attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_host", "attn_plan",
+        "attn_get_device_status", "attn_strerror", "attn_version"])
 
 
 def test_every_declared_symbol_is_exported():
@@ -107,7 +107,7 @@ def test_no_silent_fallback_without_device():
 
 
 def test_host_entry_argument_errors():
-    base = [0x1000] * 10
+    base = [0x1000] * 10 + [None, 0]
     args = dict(B=1, H=1, Nq=8, Nk=8, d=64, scale=0.125, causal=0, dtype=0, stream=None)
     assert A.attn_fwd_host(None, *base[1:], *args.values()) == 1
     ptrs = list(base)
@@ -117,15 +117,34 @@ def test_host_entry_argument_errors():
     assert A.attn_fwd_host(*base, *args.values()) == 3
 
 
+def test_workspace_entry_argument_errors():
+    a = dict(GOOD)
+    assert A.attn_fwd_ws(None, a["k"], a["v"], a["o"], a["lse"], 1, 2, 400, 400, 64, 0.125, 0, 0,
+                         0x60000, 1 << 20, None) == 1
+    assert A.attn_fwd_ws(a["q"], a["k"], a["v"], a["o"], a["lse"], 1, 2, 400, 400, 96, 0.125, 0,
+                         0, 0x60000, 1 << 20, None) == 3
+    with pytest.raises(A.AttnError) as e:
+        A.attn_workspace_size(1, 2, 400, 400, 80, 0)
+    assert e.value.status == 3
+
+
 def test_plan_geometry():
     p = A.attn_plan(1, 2, 400, 400, 64, 0, 148)
     assert (p["num_q_tiles"], p["num_q_pairs"], p["num_kv_tiles"], p["num_units"]) == (4, 2, 4, 4)
+    # fewer units than SMs: split mode spreads the 4 x 4 (unit, key tile) steps over 16 CTAs
+    assert (p["split"], p["split_grid"]) == (1, 16) and p["workspace_bytes"] > 0
     assert p["grid"] == 4 and p["block"] == 384
     assert p["qk_tile_products"] == 2 * 4 * 4
     p = A.attn_plan(16, 4, 1600, 1600, 64, 0, 148)
     assert (p["num_q_tiles"], p["num_q_pairs"], p["num_units"], p["grid"]) == (13, 7, 448, 148)
+    # 448 units on 148 SMs leave a ragged fourth wave: split
+    assert (p["split"], p["split_grid"]) == (1, 148)
+    assert p["workspace_bytes"] == 148 * 2 * 2 * 128 * 65 * 4 + 448 * 4 + 16
+    p3 = A.attn_plan(16, 4, 6400, 6400, 64, 0, 148)  # 1600 units: 98 % even already
+    assert p3["split"] == 0 and p3["workspace_bytes"] == 0
     assert p["smem_bytes"] <= 232448
     p = A.attn_plan(32, 16, 2048, 2048, 64, 1, 148)
+    assert p["split"] == 0  # causal work is balanced by the mirror pairing instead
     # causal: a unit is a heavy query pair with its mirror (8 pairs -> 4 units per head)
     assert (p["num_q_pairs"], p["units_per_head"], p["num_units"]) == (8, 4, 32 * 16 * 4)
     # causal: query tile i visits key tiles 0..i

@@ -249,3 +249,88 @@ def test_device_errors_do_not_launch():
     st = A.attn_fwd(base, base, base, base, None, 1, 1, 8, 8, 80, 0.1, 0, 0, 0)
     assert st == 3
     assert A.attn_get_device_status()[0] == 0
+
+
+# ------------------------------------------------------------ split mode (attn_fwd_ws)
+
+def _run_ws(q, k, v, causal, scale):
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    ws = A.workspace_for(qd, kd, causal)
+    o, lse = A.forward(qd, kd, vd, causal=causal, scale=scale, workspace=ws)
+    torch.cuda.synchronize()
+    st, word = A.attn_get_device_status()
+    assert st == 0, f"device status {word:#x}"
+    return o.cpu(), lse.cpu(), ws
+
+
+@pytest.mark.parametrize("idx", [0, 1])
+def test_split_workloads(idx):
+    """The YOLO 20x20 and 40x40 workloads run in split mode and match the oracle."""
+    w = WORKLOADS[idx]
+    q, k, v = make_workload_qkv(w)
+    o, lse, ws = _run_ws(q, k, v, w.causal, w.scale)
+    assert ws is not None, "split mode expected for this workload"
+    o_ref, l_ref = oracle.attention_f64(q, k, v, w.scale, w.causal)
+    assert _err(o.double().numpy(), o_ref) <= TOL[w.dtype]
+    assert _err(lse.double().numpy(), l_ref) <= LSE_TOL
+
+
+@pytest.mark.parametrize("B,H,Nq,Nk,d,dtype", [
+    (1, 1, 2000, 2000, 64, "fp16"),    # 8 units x 16 key tiles on 128 CTAs: 16 pieces per unit
+    (1, 1, 1000, 1700, 128, "bf16"),   # ragged keys, 14 pieces per unit
+    (1, 3, 300, 900, 64, "bf16"),      # odd query tiles: tile 1 of the last pair is empty
+    (2, 1, 129, 257, 128, "fp16"),
+])
+def test_split_many_pieces(B, H, Nq, Nk, d, dtype):
+    q, k, v = make_qkv(B, H, Nq, Nk, d, dtype, seed=Nq + Nk + d)
+    scale = 1.0 / math.sqrt(d)
+    o, lse, ws = _run_ws(q, k, v, False, scale)
+    assert ws is not None
+    o_ref, l_ref = oracle.attention_f64(q, k, v, scale, False)
+    assert _err(o.double().numpy(), o_ref) <= TOL[dtype]
+    assert _err(lse.double().numpy(), l_ref) <= LSE_TOL
+
+
+def test_split_workspace_reuse_is_deterministic():
+    """Reusing one workspace gives the same bits: each call leaves the counters at zero."""
+    q, k, v = (t.cuda() for t in make_qkv(1, 2, 1500, 1500, 64, "fp16", seed=31))
+    ws = A.workspace_for(q, k, False)
+    o1, l1 = A.forward(q, k, v, workspace=ws)
+    o2, l2 = A.forward(q, k, v, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    o3, l3 = A.forward(q, k, v)  # unsplit
+    torch.cuda.synchronize()
+    n_units = A.attn_plan(1, 2, 1500, 1500, 64, 0, 148)["num_units"]
+    counters = ws[-(n_units * 4 + 16):-16].view(torch.int32)
+    assert int(counters.abs().sum()) == 0
+    assert _err(o1.cpu().double().numpy(), o3.cpu().double().numpy()) <= TOL["fp16"]
+    assert _err(l1.cpu().double().numpy(), l3.cpu().double().numpy()) <= LSE_TOL
+
+
+def test_split_small_workspace_falls_back_to_units():
+    """A workspace that is too small is ignored (same as attn_fwd), not overrun."""
+    q, k, v = (t.cuda() for t in make_qkv(1, 2, 400, 400, 64, "fp16", seed=32))
+    small = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    o1, l1 = A.forward(q, k, v, workspace=small)
+    o2, l2 = A.forward(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    assert int(small.sum()) == 0
+
+
+def test_host_entry_with_workspace():
+    w = WORKLOADS[1]
+    q, k, v = make_workload_qkv(w)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32).pin_memory()
+    qd, kd, vd = (torch.empty_like(t, device="cuda") for t in (q, k, v))
+    od = torch.empty_like(qd)
+    ld = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device="cuda")
+    ws = A.workspace_for(qd, kd, w.causal)
+    A.forward_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, causal=w.causal, workspace=ws)
+    torch.cuda.synchronize()
+    o, lse = A.forward(q.cuda(), k.cuda(), v.cuda(), causal=w.causal, workspace=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, o.cpu()) and torch.equal(lh, lse.cpu())
