@@ -22,6 +22,7 @@ __all__ = [
     "ATTN_FP16", "ATTN_BF16", "AttnError", "lib", "library_path", "attn_fwd", "attn_fwd_host",
     "attn_plan", "attn_get_device_status", "attn_strerror", "attn_version", "forward",
     "forward_host", "STATUS_NAMES", "attn_fwd_ws", "attn_workspace_size", "workspace_for",
+    "attn_fwd_noalloc",
 ]
 
 ATTN_FP16 = 0
@@ -29,7 +30,7 @@ ATTN_BF16 = 1
 STATUS_NAMES = {
     0: "ATTN_OK", 1: "ATTN_ERR_NULL", 2: "ATTN_ERR_SHAPE", 3: "ATTN_ERR_HEAD_DIM",
     4: "ATTN_ERR_DTYPE", 5: "ATTN_ERR_ALIGN", 6: "ATTN_ERR_SCALE", 7: "ATTN_ERR_ARCH",
-    8: "ATTN_ERR_CUDA", 9: "ATTN_ERR_DEVICE_TIMEOUT",
+    8: "ATTN_ERR_CUDA", 9: "ATTN_ERR_DEVICE_TIMEOUT", 10: "ATTN_ERR_SCRATCH_LIMIT",
 }
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -78,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_ws.restype = i
         L.attn_workspace_size.argtypes = [i, i, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
         L.attn_workspace_size.restype = i
+        L.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
+        L.attn_fwd_noalloc.restype = i
         L.attn_fwd_host.argtypes = [vp] * 11 + [ctypes.c_size_t, i, i, i, i, i, f, i, i, vp]
         L.attn_fwd_host.restype = i
         L.attn_plan.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(_Plan)]
@@ -104,6 +107,15 @@ def attn_fwd_ws(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, workspac
     """Raw ``attn_fwd_ws``: attn_fwd with a device workspace (split mode)."""
     return lib().attn_fwd_ws(q, k, v, o, lse, B, H, Nq, Nk, d, float(scale), int(causal), dtype,
                              workspace, ws_bytes, stream)
+
+
+def attn_fwd_noalloc(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, stream) -> int:
+    """Raw ``attn_fwd_noalloc``: split mode with the library's fixed scratch, no allocation.
+
+    For callers that cannot allocate device memory themselves (see include/attn.h).
+    """
+    return lib().attn_fwd_noalloc(q, k, v, o, lse, B, H, Nq, Nk, d, float(scale), int(causal),
+                                  dtype, stream)
 
 
 def attn_workspace_size(B, H, Nq, Nk, d, causal) -> int:

@@ -394,10 +394,84 @@ const char* attn_strerror(int status) {
     case ATTN_ERR_ARCH: return "the current device is not compute capability 10.0 (sm_100a)";
     case ATTN_ERR_CUDA: return "a CUDA call failed (no usable device, encode or launch error)";
     case ATTN_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded internal wait; its output is invalid";
+    case ATTN_ERR_SCRATCH_LIMIT: return "the problem needs more scratch than attn_fwd_noalloc's fixed 24 MiB";
     default: return "unknown status";
   }
 }
 
 int attn_version(void) { return 100; }
+
+}  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free entry point.
+//
+// Some callers cannot allocate device memory at all: a plugin running inside
+// a framework that owns every byte of device memory through its own
+// allocator, a deployment whose memory plan is fixed before it starts, or a
+// latency-critical path where cudaMalloc's implicit device synchronisation
+// would stall other streams.  For them attn_fwd_noalloc takes its split-mode
+// workspace from the fixed array below instead of from the caller.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 24u << 20;  // 24 MiB
+
+// Split-mode workspace of attn_fwd_noalloc.  Every GPU that loads this library
+// holds these 24 MiB until the process exits.  In host code the name is only
+// a stand-in: the device address comes from cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+void* g_noalloc_ptr[kMaxDevices] = {};  // device address per device, guarded by g_dev_mutex
+
+// First call on a device: look up the array's device address with that device
+// current (this is why the first call should come before any stream capture).
+int noalloc_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_noalloc_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    g_noalloc_ptr[dev] = ptr;
+  }
+  *out = g_noalloc_ptr[dev];
+  return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                                int B, int H, int Nq, int Nk, int d, float scale, int causal,
+                                int dtype, attn_stream_t stream) {
+  int st = check_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, dtype);
+  if (st != ATTN_OK) return st;
+  int dev = -1;
+  DeviceInfo* info = nullptr;
+  st = current_device(&dev, &info);
+  if (st != ATTN_OK) return st;
+  attn_plan_t plan;
+  fill_plan(B, H, Nq, Nk, d, causal, info->sms, &plan);
+  if (!plan.split)  // this shape needs no scratch at all
+    return fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, nullptr, 0, stream);
+  if (static_cast<size_t>(plan.workspace_bytes) > kNoAllocScratchBytes) return ATTN_ERR_SCRATCH_LIMIT;
+  void* ws = nullptr;
+  st = noalloc_scratch(dev, &ws);
+  if (st != ATTN_OK) return st;
+  // The array keeps the previous call's contents; the piece counters must
+  // start at zero (a call that timed out may have left them set).
+  const size_t rows = static_cast<size_t>(plan.split_grid) * 2 * 2 * BLOCK_M;
+  char* counters = static_cast<char*>(ws) + rows * (d + 1) * sizeof(float);
+  if (cudaMemsetAsync(counters, 0, static_cast<size_t>(plan.num_units) * 4,
+                      reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  return fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, ws,
+                  kNoAllocScratchBytes, stream);
+}
+
+extern "C" {
 
 }  // extern "C"

@@ -52,7 +52,8 @@ typedef enum {
   ATTN_ERR_SCALE = 6,          /* scale is not finite and > 0 */
   ATTN_ERR_ARCH = 7,           /* current device is not compute capability 10.0 (B200) */
   ATTN_ERR_CUDA = 8,           /* a CUDA runtime / driver call failed (no device, launch error) */
-  ATTN_ERR_DEVICE_TIMEOUT = 9  /* a kernel gave up waiting (see attn_get_device_status) */
+  ATTN_ERR_DEVICE_TIMEOUT = 9, /* a kernel gave up waiting (see attn_get_device_status) */
+  ATTN_ERR_SCRATCH_LIMIT = 10   /* attn_fwd_noalloc: the problem needs more than its fixed scratch */
 } attn_status_t;
 
 /* Launch geometry for one call (see attn_plan). */
@@ -131,6 +132,34 @@ int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse
  * ATTN_ERR_HEAD_DIM, ATTN_ERR_SHAPE, ATTN_ERR_CUDA / ATTN_ERR_ARCH (no usable device).
  */
 int attn_workspace_size(int B, int H, int Nq, int Nk, int d, int causal, size_t* bytes);
+
+/*
+ * attn_fwd_noalloc -- attn_fwd_ws without a caller workspace and without any allocation.
+ *
+ * The pages have no counterpart to this entry point; it exists for callers that cannot
+ * allocate device memory: a plugin inside a framework that owns all device memory through
+ * its own allocator, a deployment whose memory plan is fixed before it runs, or a path where
+ * cudaMalloc's implicit device-wide synchronisation would stall other work.  It computes
+ * exactly what attn_fwd_ws computes (same kernel, split mode where that pays) but takes the
+ * workspace from a fixed 24 MiB array inside the library.  Every GPU that loads the library
+ * holds that array until the process exits.
+ *
+ *   - Arguments, layouts and the other error codes as attn_fwd.  Nothing is allocated: no
+ *     cudaMalloc, no cudaFree, no allocating library call.
+ *   - Returns ATTN_ERR_SCRATCH_LIMIT, without enqueueing anything, when split mode would need
+ *     more than 24 MiB of scratch (at d = 64 every split plan on a 148-SM B200 fits; at
+ *     d = 128 split plans of more than about 94 CTAs do not -- use attn_fwd_ws for those).
+ *     Shapes that need no split mode never touch the array and are never rejected.
+ *   - The first call on a device looks up the array's device address with that device
+ *     current; make that first call before any stream capture.
+ *   - Every call shares the one array and it keeps the previous call's contents; each call
+ *     clears the part that must start at zero (a memset on `stream`).  Calls whose execution
+ *     overlaps on the GPU (different streams, different host threads, no ordering between
+ *     them) race on the array and may return wrong results: order them.
+ */
+int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                     int H, int Nq, int Nk, int d, float scale, int causal, int dtype,
+                     attn_stream_t stream);
 
 /*
  * attn_fwd_host -- the same forward, end to end from host memory.

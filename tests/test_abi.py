@@ -33,8 +33,8 @@ def header_functions():
 
 def test_header_declares_the_boundary():
     assert header_functions() == sorted([
-        "attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_host", "attn_plan",
-        "attn_get_device_status", "attn_strerror", "attn_version"])
+        "attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_noalloc", "attn_fwd_host",
+        "attn_plan", "attn_get_device_status", "attn_strerror", "attn_version"])
 
 
 def test_every_declared_symbol_is_exported():
@@ -54,8 +54,8 @@ def test_status_enum_matches_header():
 
 
 def test_strerror_and_version():
-    for code in range(10):
-        assert A.attn_strerror(code)
+    for code in range(11):
+        assert A.attn_strerror(code) != "unknown status"
     assert A.attn_strerror(1234) == "unknown status"
     assert A.attn_version() == 100
 
