@@ -81,6 +81,9 @@ def lib() -> ctypes.CDLL:
         L.attn_workspace_size.restype = i
         L.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
         L.attn_fwd_noalloc.restype = i
+        L.attn_fwd_stall_test.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp,
+                                          ctypes.c_size_t, i, vp]
+        L.attn_fwd_stall_test.restype = i
         L.attn_fwd_host.argtypes = [vp] * 11 + [ctypes.c_size_t, i, i, i, i, i, f, i, i, vp]
         L.attn_fwd_host.restype = i
         L.attn_plan.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(_Plan)]
@@ -116,6 +119,13 @@ def attn_fwd_noalloc(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, str
     """
     return lib().attn_fwd_noalloc(q, k, v, o, lse, B, H, Nq, Nk, d, float(scale), int(causal),
                                   dtype, stream)
+
+
+def attn_fwd_stall_test(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, workspace,
+                        ws_bytes, stall_site, stream) -> int:
+    """Raw ``attn_fwd_stall_test``: the failure-path test hook (see include/attn.h)."""
+    return lib().attn_fwd_stall_test(q, k, v, o, lse, B, H, Nq, Nk, d, float(scale),
+                                     int(causal), dtype, workspace, ws_bytes, stall_site, stream)
 
 
 def attn_workspace_size(B, H, Nq, Nk, d, causal) -> int:

@@ -225,7 +225,8 @@ int launch(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo& inf
 
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                     int H, int Nq, int Nk, int d, float scale, int causal, int dtype,
-                    void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+                    void* workspace, size_t workspace_bytes, attn_stream_t stream,
+                    int stall_site = 0) {
   int st = check_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, dtype);
   if (st != ATTN_OK) return st;
   int dev = -1;
@@ -265,6 +266,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   prm.ws_o = nullptr;
   prm.ws_lse = nullptr;
   prm.ws_count = nullptr;
+  prm.stall_site = stall_site;
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int grid = plan.grid;
@@ -303,6 +305,15 @@ int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse
                 size_t workspace_bytes, attn_stream_t stream) {
   return fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, workspace,
                   workspace_bytes, stream);
+}
+
+int attn_fwd_stall_test(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int H, int Nq, int Nk, int d, float scale, int causal, int dtype,
+                        void* workspace, size_t workspace_bytes, int stall_site,
+                        attn_stream_t stream) {
+  if (stall_site < 1 || stall_site > 4) return ATTN_ERR_SHAPE;
+  return fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, workspace,
+                  workspace_bytes, stream, stall_site);
 }
 
 int attn_workspace_size(int B, int H, int Nq, int Nk, int d, int causal, size_t* bytes) {

@@ -87,6 +87,17 @@ enum WaitSite : uint32_t {
   SITE_SOFTMAX_S_FULL = 6,
   SITE_SOFTMAX_O_READY = 7,
   SITE_DRAIN = 8,
+  SITE_SOFTMAX_SYNC = 9,
+  SITE_INJECTED = 10,  // a wait made unsatisfiable on purpose (attn_fwd_stall_test)
+};
+
+// Test hook: which role waits on a barrier nothing ever arrives on.
+enum StallSite : int {
+  STALL_NONE = 0,
+  STALL_SOFTMAX = 1,     // softmax warpgroup 0, before its first score tile
+  STALL_MMA = 2,         // the S-issuing MMA warp, before its first MMA
+  STALL_LOAD = 3,        // the K/Q TMA warp, before its first load
+  STALL_SPLIT_SYNC = 4,  // softmax warpgroup 0, before the split-piece rendezvous
 };
 
 struct FwdParams {
@@ -110,6 +121,7 @@ struct FwdParams {
   float* ws_o;           // [grid][2 slots][2 tiles][128 rows][D]
   float* ws_lse;         // [grid][2 slots][2 tiles][128 rows]
   unsigned int* ws_count;  // [num_units] pieces finished; zero between calls
+  int stall_site;          // StallSite; 0 except through the test hook
 };
 
 template <int D>
@@ -143,7 +155,9 @@ struct SmemLayout {
   static constexpr int O_READY = P_FULL + NSB; // + tile: one phase per P V MMA of the tile
   static constexpr int PV_DONE = O_READY + 2;  // + buffer: P V of that buffer finished
   static constexpr int DRAIN = PV_DONE + NSB;  // + 0 (S warp), + 1 (P V warp)
-  static constexpr int NUM_BARS = DRAIN + 2;
+  static constexpr int SYNC = DRAIN + 2;        // rendezvous of the 256 softmax threads
+  static constexpr int NEVER = SYNC + 1;        // no thread ever arrives (test hook)
+  static constexpr int NUM_BARS = NEVER + 1;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // TMEM address, abort flag
   static constexpr int BYTES = MISC_OFF + 16 + 1024;      // + slack to align the base to 1 KB
   // TMEM columns (512 allocated): S/P buffers, then O of tile 0 and tile 1
@@ -280,9 +294,6 @@ __device__ __forceinline__ size_t ws_o_base(int cta, int slot, int t, int D) {
   return ((static_cast<size_t>(cta) * 2 + slot) * 2 + t) * static_cast<size_t>(BLOCK_M) * D;
 }
 
-__device__ __forceinline__ void softmax_barrier() {
-  asm volatile("bar.sync 1, 256;" ::: "memory");  // the eight softmax warps only
-}
 
 // The S sequence of one item: the MMA warp computes the score tiles of the
 // two Q tiles alternately, S_0(0), S_1(0), S_0(1), S_1(1), ..., and, when
@@ -368,6 +379,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int b = 0; b < NSB; ++b) mbar_init(bar(L::PV_DONE + b), 1);
     mbar_init(bar(L::DRAIN + 0), 1);
     mbar_init(bar(L::DRAIN + 1), 1);
+    mbar_init(bar(L::SYNC), 2 * 128);
+    mbar_init(bar(L::NEVER), 1);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -419,6 +432,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       while (ok && cur.next(p, w)) {
         {
           if (is_k) {
+            if (p.stall_site == STALL_LOAD) {
+              warp_wait(bar(L::NEVER), 0, SITE_INJECTED);
+              ok = false;
+              break;
+            }
             if (items_done > 0) {
               ok = warp_wait(bar(L::Q_EMPTY), (items_done - 1) & 1, SITE_LOAD_Q_EMPTY);
               if (!ok) break;
@@ -505,6 +523,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         {
           const int total = w.n[0] + w.n[1];
           if (is_s) {
+            if (p.stall_site == STALL_MMA) {
+              warp_wait(bar(L::NEVER), 0, SITE_INJECTED);
+              ok = false;
+              break;
+            }
             ok = warp_wait(bar(L::Q_FULL), q_phase, SITE_MMA_Q_FULL);
             if (!ok) break;
             q_phase ^= 1;
@@ -664,6 +687,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t s_parity = 0;  // bit b: parity of the next S_FULL(b, t) phase this warpgroup waits for
     bool ok = true;
     volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
+    uint32_t sync_phase = 0;
+    auto softmax_sync = [&]() -> bool {
+      mbar_arrive(bar(L::SYNC));
+      const bool r = wait_phase(bar(L::SYNC), sync_phase, abort_flag, SITE_SOFTMAX_SYNC);
+      sync_phase ^= 1;
+      return __all_sync(0xffffffffu, r);
+    };
     WorkCursor<SPLIT> cur(p);
     Unit w;
     while (ok && cur.next(p, w)) {
@@ -681,6 +711,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t kg = item_sk + seq_pos(w, t, j);
           const uint32_t b = kg % NSB;
           const uint32_t tS = tS0 + 128 * b;
+          if (p.stall_site == STALL_SOFTMAX && t == 0) {
+            wait_phase(bar(L::NEVER), 0, abort_flag, SITE_INJECTED);
+            ok = false;
+            break;
+          }
           ok = wait_phase(bar(L::S_FULL + 2 * b + t), (s_parity >> b) & 1u, abort_flag,
                           SITE_SOFTMAX_S_FULL);
           ok = __all_sync(0xffffffffu, ok);
@@ -847,17 +882,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // them with the log-domain identity lse = ln sum_k e^{lse_k},
           // O = sum_k e^{lse_k - lse} O_k, and resets the counter for the
           // next call.
+          // The two rendezvous are bounded mbarrier waits, not bar.sync: if
+          // the other warpgroup has aborted, this one gives up too instead
+          // of waiting forever.  (The flag is rewritten only after the next
+          // item's first rendezvous, which every thread reaches after
+          // reading it.)
           __threadfence();
-          softmax_barrier();
+          if (p.stall_site == STALL_SPLIT_SYNC && t == 0) {
+            wait_phase(bar(L::NEVER), 0, abort_flag, SITE_INJECTED);
+            break;
+          }
+          if (!softmax_sync()) break;
           if (threadIdx.x == 0) {
             const unsigned int done = atomicAdd(p.ws_count + w.unit, 1u);
             const int last = (done == static_cast<unsigned int>(w.pieces - 1)) ? 1 : 0;
             if (last) p.ws_count[w.unit] = 0u;
             *last_flag = last;
           }
-          softmax_barrier();
+          if (!softmax_sync()) break;
           const bool last = *last_flag != 0;
-          softmax_barrier();  // everyone has read the flag before it is reused
           const int n_unit = t ? (w.q0 + BLOCK_M < p.Nq) : 1;  // does tile t have rows at all
           if (last && n_unit) {
             // This CTA finished the unit's last piece.  Its own piece is still

@@ -162,6 +162,27 @@ int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float
                      attn_stream_t stream);
 
 /*
+ * attn_fwd_stall_test -- test hook for the failure path; not for production use.
+ *
+ * Enqueues attn_fwd_ws (same arguments) with one internal wait pointed at a barrier that
+ * nothing ever arrives on, so that the bounded wait runs out after about one second:
+ *   stall_site 1: softmax warpgroup 0, before its first score tile;
+ *              2: the MMA warp, before its first MMA;
+ *              3: the Q/K TMA warp, before its first load;
+ *              4: softmax warpgroup 0, before the split-piece rendezvous (split mode only).
+ * The kernel records 0x8000000A in the device status word, every role leaves its loop, the
+ * issued loads and MMAs are waited for, tensor memory is freed and the kernel returns;
+ * attn_get_device_status() then reports ATTN_ERR_DEVICE_TIMEOUT and the CUDA context stays
+ * usable.  o / lse hold no meaningful result; a split-mode workspace must be zero-filled
+ * again afterwards.  Returns ATTN_ERR_SHAPE for a stall_site outside 1..4, otherwise the
+ * codes of attn_fwd_ws.  Nothing here faults or traps the GPU.
+ */
+int attn_fwd_stall_test(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                        int H, int Nq, int Nk, int d, float scale, int causal, int dtype,
+                        void* workspace, size_t workspace_bytes, int stall_site,
+                        attn_stream_t stream);
+
+/*
  * attn_fwd_host -- the same forward, end to end from host memory.
  *
  * Enqueues on `stream`: host->device copies of q_host, k_host, v_host into the caller's

@@ -34,7 +34,8 @@ def header_functions():
 def test_header_declares_the_boundary():
     assert header_functions() == sorted([
         "attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_noalloc", "attn_fwd_host",
-        "attn_plan", "attn_get_device_status", "attn_strerror", "attn_version"])
+        "attn_fwd_stall_test", "attn_plan", "attn_get_device_status", "attn_strerror",
+        "attn_version"])
 
 
 def test_every_declared_symbol_is_exported():
