@@ -229,17 +229,34 @@ __device__ __forceinline__ Unit decode_item(const FwdParams& p, int u, int item)
 template <bool SPLIT>
 struct WorkCursor {
   int u, item, items;
-  long long idx, end;
+  // split mode: this CTA's units u .. u_last, the first starting at key tile
+  // j_first, the last ending before key tile j_end; pieces of the first and
+  // last unit (every unit in between lies wholly inside the range)
+  int u_last, j_first, j_end;
+  int piece_first, pieces_first, c_first_first;
+  int piece_last, pieces_last, c_first_last;
   __device__ __forceinline__ explicit WorkCursor(const FwdParams& p) {
     if constexpr (SPLIT) {
-      idx = p.total_steps * blockIdx.x / gridDim.x;
-      end = p.total_steps * (blockIdx.x + 1) / gridDim.x;
-      u = item = items = 0;
+      // the 64-bit divisions run once per CTA, not once per item
+      const long long begin = p.total_steps * blockIdx.x / gridDim.x;
+      const long long end = p.total_steps * (blockIdx.x + 1) / gridDim.x;
+      const int nk = p.num_kv_tiles;
+      item = items = 0;
+      if (begin >= end) {
+        u = 0;
+        u_last = -1;
+        return;
+      }
+      u = static_cast<int>(begin / nk);
+      j_first = static_cast<int>(begin - static_cast<long long>(u) * nk);
+      u_last = static_cast<int>((end - 1) / nk);
+      j_end = static_cast<int>(end - static_cast<long long>(u_last) * nk);
+      pieces_of(p, u, j_first, piece_first, pieces_first, c_first_first);
+      pieces_of(p, u_last, 0, piece_last, pieces_last, c_first_last);
     } else {
       u = blockIdx.x;
       item = 0;
       items = u < p.num_units ? unit_items(p, u) : 0;
-      idx = end = 0;
     }
   }
   // Number of CTAs c >= 1 whose step range begins at or before step x.
@@ -248,25 +265,44 @@ struct WorkCursor {
     const long long c = ((x + 1) * g - 1) / p.total_steps;
     return c < g - 1 ? c : g - 1;
   }
+  // Piece index of the part of unit uu starting at key tile j0, the unit's
+  // number of pieces, and the CTA holding piece 0.
+  __device__ __forceinline__ static void pieces_of(const FwdParams& p, int uu, int j0, int& piece,
+                                                   int& pieces, int& c_first) {
+    const int nk = p.num_kv_tiles;
+    const long long a = static_cast<long long>(uu) * nk;
+    const long long ca = starts_le(p, a);
+    piece = static_cast<int>(starts_le(p, a + j0) - ca);
+    pieces = static_cast<int>(1 + starts_le(p, a + nk - 1) - ca);
+    c_first = static_cast<int>(ca);
+  }
   __device__ __forceinline__ bool next(const FwdParams& p, Unit& w) {
     if constexpr (SPLIT) {
-      if (idx >= end) return false;
+      if (u > u_last) return false;
       const int nk = p.num_kv_tiles;
-      const int uu = static_cast<int>(idx / nk);
-      const int j0 = static_cast<int>(idx % nk);
-      const long long left = end - idx;
-      const int j1 = left < nk - j0 ? j0 + static_cast<int>(left) : nk;
-      w = decode_item(p, uu, 0);
+      const bool first = (item == 0);
+      const int j0 = first ? j_first : 0;
+      const int j1 = (u == u_last) ? j_end : nk;
+      w = decode_item(p, u, 0);
       w.jbase = j0;
       w.n[0] = w.n[0] > 0 ? j1 - j0 : 0;
       w.n[1] = w.n[1] > 0 ? j1 - j0 : 0;
       w.nmax = max(w.n[0], w.n[1]);
-      const long long a = static_cast<long long>(uu) * nk;
-      const long long ca = starts_le(p, a);
-      w.piece = static_cast<int>(starts_le(p, a + j0) - ca);
-      w.pieces = static_cast<int>(1 + starts_le(p, a + nk - 1) - ca);
-      w.c_first = static_cast<int>(ca);
-      idx += j1 - j0;
+      if (first) {
+        w.piece = piece_first;
+        w.pieces = pieces_first;
+        w.c_first = c_first_first;
+      } else if (u == u_last) {
+        w.piece = piece_last;
+        w.pieces = pieces_last;
+        w.c_first = c_first_last;
+      } else {
+        w.piece = 0;
+        w.pieces = 1;
+        w.c_first = static_cast<int>(blockIdx.x);
+      }
+      item = 1;
+      ++u;
       return true;
     } else {
       while (item >= items) {
