@@ -54,11 +54,11 @@ class AttnError(RuntimeError):
 class _Plan(ctypes.Structure):
     _fields_ = [("num_q_tiles", ctypes.c_int), ("num_q_pairs", ctypes.c_int),
                 ("num_kv_tiles", ctypes.c_int), ("units_per_head", ctypes.c_int),
-                ("num_units", ctypes.c_int),
+                ("num_units", ctypes.c_int), ("dual_units", ctypes.c_int),
                 ("grid", ctypes.c_int), ("block", ctypes.c_int), ("smem_bytes", ctypes.c_int),
                 ("stages", ctypes.c_int), ("qk_tile_products", ctypes.c_longlong),
                 ("split", ctypes.c_int), ("split_grid", ctypes.c_int),
-                ("workspace_bytes", ctypes.c_longlong)]
+                ("split_units", ctypes.c_int), ("workspace_bytes", ctypes.c_longlong)]
 
 
 def lib() -> ctypes.CDLL:

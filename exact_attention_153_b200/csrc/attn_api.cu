@@ -50,7 +50,7 @@ struct DeviceInfo {
   bool probed = false;
   bool supported = false;
   int sms = 0;
-  bool smem_attr[2][2][2] = {};  // [d==128][bf16][split]
+  bool smem_attr[2][2][3] = {};  // [d==128][bf16][unit, dual-unit, split kernel]
 };
 
 std::mutex g_dev_mutex;
@@ -102,13 +102,19 @@ void fill_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, att
   const int q_tiles = ceil_div(Nq, BLOCK_M);
   const int q_pairs = ceil_div(q_tiles, 2);
   const int kv_tiles = ceil_div(Nk, BLOCK_N);
-  const int units_per_head = causal ? (q_pairs + 1) / 2 : q_pairs;
-  const long long units = static_cast<long long>(B) * H * units_per_head;
+  const long long BH = static_cast<long long>(B) * H;
+  // Unit mode pairs the lone last query tile of two heads into one dual unit
+  // when the tile count is odd (non-causal), so no warpgroup idles.
+  const bool dual = !causal && (q_tiles % 2 == 1) && BH >= 2;
+  const int units_per_head = causal ? (q_pairs + 1) / 2 : (dual ? q_tiles / 2 : q_pairs);
+  const long long dual_units = dual ? (BH + 1) / 2 : 0;
+  const long long units = BH * units_per_head + dual_units;
   out->num_q_tiles = q_tiles;
   out->num_q_pairs = q_pairs;
   out->num_kv_tiles = kv_tiles;
   out->num_units = static_cast<int>(units);
   out->units_per_head = units_per_head;
+  out->dual_units = static_cast<int>(dual_units);
   out->grid = static_cast<int>(units < num_sms ? units : num_sms);
   out->block = NUM_THREADS;
   out->smem_bytes = d == 64 ? SmemLayout<64>::BYTES : SmemLayout<128>::BYTES;
@@ -126,11 +132,14 @@ void fill_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, att
     }
   }
   out->qk_tile_products = per_head * B * H;
-  const long long total_steps = units * kv_tiles;
-  out->split = split_pays(units, total_steps, num_sms, causal) ? 1 : 0;
+  // split mode keeps plain units (one (batch, head) each): q_pairs per head
+  const long long split_units = BH * q_pairs;
+  const long long total_steps = split_units * kv_tiles;
+  out->split = (!causal && split_pays(units, total_steps, num_sms, causal)) ? 1 : 0;
   out->split_grid = static_cast<int>(total_steps < num_sms ? total_steps : num_sms);
+  out->split_units = static_cast<int>(split_units);
   out->workspace_bytes =
-      out->split ? static_cast<long long>(split_workspace_bytes(out->split_grid, d, units)) : 0;
+      out->split ? static_cast<long long>(split_workspace_bytes(out->split_grid, d, split_units)) : 0;
 }
 
 // Probe the current device once: compute capability 10.0 and SM count.
@@ -193,12 +202,12 @@ struct MapCache {
 };
 thread_local MapCache t_maps;
 
-template <int D, bool BF16, bool SPLIT>
+template <int D, bool BF16, bool SPLIT, bool DUAL>
 int launch_one(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo& info,
                cudaStream_t stream) {
-  auto kernel = attn_sm100::attn_fwd_kernel<D, BF16, SPLIT>;
+  auto kernel = attn_sm100::attn_fwd_kernel<D, BF16, SPLIT, DUAL>;
   constexpr int smem = SmemLayout<D>::BYTES;
-  bool& attr = info.smem_attr[D == 128][BF16][SPLIT];
+  bool& attr = info.smem_attr[D == 128][BF16][SPLIT ? 2 : (DUAL ? 1 : 0)];
   if (!attr) {
     std::lock_guard<std::mutex> lock(g_dev_mutex);
     if (!attr) {
@@ -214,13 +223,14 @@ int launch_one(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo&
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }
 
-// Split mode is a separate instantiation, so the unit-mode kernel carries none
-// of the piece bookkeeping.
+// Split mode and unit mode with dual units are separate instantiations, so
+// the plain unit-mode kernel carries none of their bookkeeping.
 template <int D, bool BF16>
 int launch(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo& info,
            cudaStream_t stream) {
-  return prm.split ? launch_one<D, BF16, true>(maps, prm, grid, info, stream)
-                   : launch_one<D, BF16, false>(maps, prm, grid, info, stream);
+  if (prm.split) return launch_one<D, BF16, true, false>(maps, prm, grid, info, stream);
+  if (prm.dual_base >= 0) return launch_one<D, BF16, false, true>(maps, prm, grid, info, stream);
+  return launch_one<D, BF16, false, false>(maps, prm, grid, info, stream);
 }
 
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
@@ -259,6 +269,8 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   prm.num_kv_tiles = plan.num_kv_tiles;
   prm.units_per_head = plan.units_per_head;
   prm.num_units = plan.num_units;
+  prm.dual_base = plan.dual_units > 0 ? plan.num_units - plan.dual_units : -1;
+  prm.last_q0 = (plan.num_q_tiles - 1) * BLOCK_M;
   prm.causal = causal ? 1 : 0;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   prm.split = 0;
@@ -277,7 +289,11 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
     const size_t rows = static_cast<size_t>(grid) * 2 * 2 * BLOCK_M;
     char* ws = static_cast<char*>(workspace);
     prm.split = 1;
-    prm.total_steps = static_cast<long long>(plan.num_units) * plan.num_kv_tiles;
+    // split mode walks plain units: one (batch, head) and query pair each
+    prm.units_per_head = plan.num_q_pairs;
+    prm.num_units = plan.split_units;
+    prm.dual_base = -1;
+    prm.total_steps = static_cast<long long>(plan.split_units) * plan.num_kv_tiles;
     prm.ws_o = reinterpret_cast<float*>(ws);
     prm.ws_lse = reinterpret_cast<float*>(ws + rows * d * sizeof(float));
     // the piece counters start at zero (the caller zero-fills a new
@@ -474,7 +490,7 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
   // start at zero (a call that timed out may have left them set).
   const size_t rows = static_cast<size_t>(plan.split_grid) * 2 * 2 * BLOCK_M;
   char* counters = static_cast<char*>(ws) + rows * (d + 1) * sizeof(float);
-  if (cudaMemsetAsync(counters, 0, static_cast<size_t>(plan.num_units) * 4,
+  if (cudaMemsetAsync(counters, 0, static_cast<size_t>(plan.split_units) * 4,
                       reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;

@@ -106,8 +106,13 @@ struct FwdParams {
   int Nq, Nk, BH;
   int num_q_pairs;  // ceil(ceil(Nq / 128) / 2)
   int num_kv_tiles; // ceil(Nk / 128)
-  int units_per_head; // causal: ceil(num_q_pairs / 2); else num_q_pairs
-  int num_units;    // BH * units_per_head
+  int units_per_head; // causal: ceil(num_q_pairs / 2); dual units: num_q_tiles / 2; else num_q_pairs
+  int num_units;    // BH * units_per_head (+ the dual units)
+  // Dual units (non-causal unit mode, odd query-tile count): units from
+  // dual_base on pair the lone last query tile (rows last_q0..) of two heads;
+  // -1 when there are none.
+  int dual_base;
+  int last_q0;
   int causal;
   float scale_log2; // scale * log2(e)
   // Split mode (non-causal only).  The units' key tiles are flattened into
@@ -168,8 +173,11 @@ struct SmemLayout {
 };
 
 struct Unit {
-  int bh;
+  int bh;     // (batch, head) of tile 0
   int q0;     // first query row of tile 0
+  int bh1;    // (batch, head) of tile 1: bh, except in a dual unit
+  int q1;     // first query row of tile 1: q0 + 128, except in a dual unit
+  int kvs;    // K (and V) tiles per key step: 1 (shared by both tiles) or 2 (dual unit)
   int jbase;  // first K/V tile of this item (non-zero only for split pieces)
   int n[2];   // K/V tiles each Q tile visits from jbase (0 = tile lies past Nq)
   int nmax;
@@ -180,7 +188,11 @@ struct Unit {
 // two "items"; an item is a pair of adjacent 128-row Q tiles.  CTA c takes
 // units c, c + grid, c + 2 grid, ...; consecutive units belong to the same
 // head, so CTAs running at the same time share that head's K/V through L2.
-//   non-causal: one item per unit, every item costs the same.
+//   non-causal: one item per unit, every item costs the same.  With an odd
+//     number of query tiles each head's last tile has no partner; those
+//     tiles are paired across heads (tile 0 from head 2d, tile 1 from head
+//     2d + 1) in "dual" units placed after all the others, so no warpgroup
+//     idles through a unit.  A dual unit streams both heads' K and V.
 //   causal: unit b of a head holds Q pair (n_pairs - 1 - b) and its mirror b,
 //     heaviest first; the two together always visit about n_pairs + 1 K/V
 //     tiles, so every unit costs the same and the persistent CTAs finish
@@ -191,8 +203,26 @@ __device__ __forceinline__ int unit_items(const FwdParams& p, int u) {
   return (b != p.num_q_pairs - 1 - b) ? 2 : 1;
 }
 
+template <bool DUAL>
 __device__ __forceinline__ Unit decode_item(const FwdParams& p, int u, int item) {
   Unit w;
+  w.jbase = 0;
+  w.unit = u;
+  w.piece = 0;
+  w.pieces = 1;
+  w.c_first = 0;
+  if (DUAL && u >= p.dual_base) {
+    const int h0 = 2 * (u - p.dual_base);
+    const bool pair = h0 + 1 < p.BH;
+    w.bh = h0;
+    w.bh1 = pair ? h0 + 1 : h0;
+    w.q0 = w.q1 = p.last_q0;
+    w.n[0] = p.num_kv_tiles;
+    w.n[1] = pair ? p.num_kv_tiles : 0;
+    w.nmax = p.num_kv_tiles;
+    w.kvs = pair ? 2 : 1;
+    return w;
+  }
   int qp;
   w.bh = u / p.units_per_head;
   const int b = u % p.units_per_head;
@@ -202,6 +232,9 @@ __device__ __forceinline__ Unit decode_item(const FwdParams& p, int u, int item)
     qp = b;
   }
   w.q0 = qp * 2 * BLOCK_M;
+  w.bh1 = w.bh;
+  w.q1 = w.q0 + BLOCK_M;
+  w.kvs = 1;
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int qs = w.q0 + t * BLOCK_M;
@@ -217,16 +250,11 @@ __device__ __forceinline__ Unit decode_item(const FwdParams& p, int u, int item)
     w.n[t] = n;
   }
   w.nmax = max(w.n[0], w.n[1]);
-  w.jbase = 0;
-  w.unit = u;
-  w.piece = 0;
-  w.pieces = 1;
-  w.c_first = 0;
   return w;
 }
 
 // Iterates the items of this CTA, identically in every role.
-template <bool SPLIT>
+template <bool SPLIT, bool DUAL>
 struct WorkCursor {
   int u, item, items;
   // split mode: this CTA's units u .. u_last, the first starting at key tile
@@ -283,7 +311,7 @@ struct WorkCursor {
       const bool first = (item == 0);
       const int j0 = first ? j_first : 0;
       const int j1 = (u == u_last) ? j_end : nk;
-      w = decode_item(p, u, 0);
+      w = decode_item<false>(p, u, 0);
       w.jbase = j0;
       w.n[0] = w.n[0] > 0 ? j1 - j0 : 0;
       w.n[1] = w.n[1] > 0 ? j1 - j0 : 0;
@@ -311,7 +339,7 @@ struct WorkCursor {
         item = 0;
         items = unit_items(p, u);
       }
-      w = decode_item(p, u, item++);
+      w = decode_item<DUAL>(p, u, item++);
       return true;
     }
   }
@@ -348,10 +376,17 @@ __device__ __forceinline__ int seq_pos(const Unit& w, int t, int j) {
   const int m = min(w.n[0], w.n[1]);
   return j < m ? 2 * j + t : 2 * m + (j - m);
 }
-// K_j / V_j is used for the last time by tile 1, or by tile 0 when tile 1
-// does not visit j.
+// Ring slot (counted from the item's first) of the K or V tile that score
+// tile (t, j) uses: one per key step, or one per tile in a dual unit.
+template <bool DUAL>
+__device__ __forceinline__ int kv_slot(const Unit& w, SeqPos s) {
+  return (DUAL && w.kvs == 2) ? 2 * s.j + s.t : s.j;
+}
+// That K / V tile is used for the last time by tile 1, by tile 0 when tile 1
+// does not visit j, and always in a dual unit (each tile has its own).
+template <bool DUAL>
 __device__ __forceinline__ bool last_use(const Unit& w, SeqPos s) {
-  return s.t == 1 || s.j >= w.n[1];
+  return (DUAL && w.kvs == 2) || s.t == 1 || s.j >= w.n[1];
 }
 
 // Bounded wait on one mbarrier phase, fully inlined (a call here would make
@@ -378,7 +413,10 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
   return true;
 }
 
-template <int D, bool BF16, bool SPLIT>
+// DUAL: the unit-mode kernel for problems with dual units (an odd number of
+// query tiles per head); the other unit-mode problems run the DUAL = false
+// instantiation, which carries none of the dual-unit bookkeeping.
+template <int D, bool BF16, bool SPLIT, bool DUAL>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -463,7 +501,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const CUtensorMap* map = is_k ? &tm_k : &tm_v;
       uint32_t pos = 0, items_done = 0;
       bool ok = true;
-      WorkCursor<SPLIT> cur(p);
+      WorkCursor<SPLIT, DUAL> cur(p);
       Unit w;
       while (ok && cur.next(p, w)) {
         {
@@ -484,12 +522,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
                 for (int h = 0; h < L::HALVES; ++h)
                   tma_load_3d(q_smem + t * L::TILE_BYTES + h * L::HALF_BYTES, &tm_q,
-                              bar(L::Q_FULL), h * 64, w.q0 + t * BLOCK_M, w.bh);
+                              bar(L::Q_FULL), h * 64, (DUAL && t) ? w.q1 : w.q0 + t * BLOCK_M,
+                              (DUAL && t) ? w.bh1 : w.bh);
             }
             __syncwarp();
           }
           ++items_done;
-          for (int j = 0; ok && j < w.nmax; ++j) {
+          const int kvs = DUAL ? w.kvs : 1;
+          for (int x = 0; ok && x < w.nmax * kvs; ++x) {
+            const int j = (DUAL && kvs == 2) ? x / 2 : x;
+            const int bh = (DUAL && kvs == 2 && (x & 1)) ? w.bh1 : w.bh;
             const uint32_t st = pos % stages, ph = (pos / stages) & 1;
             if (pos >= static_cast<uint32_t>(stages) &&
                 !warp_wait(bar(empty0 + st), ph ^ 1, SITE_LOAD_KV_EMPTY)) {
@@ -501,7 +543,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
               for (int h = 0; h < L::HALVES; ++h)
                 tma_load_3d(ring + st * L::TILE_BYTES + h * L::HALF_BYTES, map, bar(full0 + st),
-                            h * 64, (w.jbase + j) * BLOCK_N, w.bh);
+                            h * 64, (w.jbase + j) * BLOCK_N, bh);
             }
             __syncwarp();
             ++pos;
@@ -553,7 +595,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t pos = 0, g = 0, q_phase = 0;  // ring position of K_0 / V_0 of the item; score tile count
       uint32_t buf = 0, round = 0;           // g % NSB, g / NSB
       bool ok = true;
-      WorkCursor<SPLIT> cur(p);
+      WorkCursor<SPLIT, DUAL> cur(p);
       Unit w;
       while (ok && cur.next(p, w)) {
         {
@@ -574,13 +616,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             int k_ready = -1, v_ready = -1;
             auto issue_s = [&](int k) -> bool {
               const SeqPos sp = seq_at(w, k);
-              const uint32_t kp = pos + sp.j;
+              const int slot = kv_slot<DUAL>(w, sp);
+              const uint32_t kp = pos + slot;
               const uint32_t st = kp % L::K_STAGES;
-              if (sp.j > k_ready) {
+              if (slot > k_ready) {
                 if (!warp_wait(bar(L::K_FULL + st), (kp / L::K_STAGES) & 1, SITE_MMA_KV_FULL))
                   return false;
                 tc_fence_after();
-                k_ready = sp.j;
+                k_ready = slot;
               }
               const uint32_t b = (g + k) % NSB;
               const uint64_t a = q_desc + static_cast<uint32_t>(sp.t * (L::TILE_BYTES >> 4));
@@ -592,21 +635,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   mma_ss(tmem_s + 128 * b, a + off, bd + off, IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(L::S_FULL + 2 * b + sp.t));
-                if (last_use(w, sp)) mma_commit(bar(L::K_EMPTY + st));
+                if (last_use<DUAL>(w, sp)) mma_commit(bar(L::K_EMPTY + st));
               }
               return true;
             };
             for (int k = 0; ok && k < min(NSB, total); ++k) ok = issue_s(k);
             for (int k = 0; ok && k < total; ++k) {
               const SeqPos sp = seq_at(w, k);
-              const uint32_t vp = pos + sp.j;
+              const int slot = kv_slot<DUAL>(w, sp);
+              const uint32_t vp = pos + slot;
               const uint32_t st = vp % L::V_STAGES;
-              if (sp.j > v_ready) {
+              if (slot > v_ready) {
                 if (!warp_wait(bar(L::V_FULL + st), (vp / L::V_STAGES) & 1, SITE_MMA_KV_FULL)) {
                   ok = false;
                   break;
                 }
-                v_ready = sp.j;
+                v_ready = slot;
               }
               const uint32_t gk = g + k;
               const uint32_t b = gk % NSB;
@@ -624,7 +668,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 // in-order issue: S_t(j + 1) completing already implies this
                 // P V completed, so only the tile's last P V is signalled
                 if (sp.j + 1 == (sp.t ? w.n[1] : w.n[0])) mma_commit(bar(L::O_READY + sp.t));
-                if (last_use(w, sp)) mma_commit(bar(L::V_EMPTY + st));
+                if (last_use<DUAL>(w, sp)) mma_commit(bar(L::V_EMPTY + st));
               }
               // the buffer of P(k) is refilled by S(k + NSB): same thread, so
               // the tensor pipe runs it after this P V
@@ -634,15 +678,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           } else
           for (int k = 0; k < total; ++k) {
             const SeqPos sp = seq_at(w, k);
+            const int slot = kv_slot<DUAL>(w, sp);
             if (is_s) {
-              const uint32_t kp = pos + sp.j;
+              const uint32_t kp = pos + slot;
               const uint32_t st = kp % L::K_STAGES;
-              if (sp.j > ready_j) {
+              if (slot > ready_j) {
                 if (!warp_wait(bar(L::K_FULL + st), (kp / L::K_STAGES) & 1, SITE_MMA_KV_FULL)) {
                   ok = false;
                   break;
                 }
-                ready_j = sp.j;
+                ready_j = slot;
               }
               if (g >= static_cast<uint32_t>(NSB) &&
                   !warp_wait(bar(L::PV_DONE + buf), (round - 1) & 1, SITE_MMA_P_FULL)) {
@@ -659,17 +704,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   mma_ss(tmem_s + 128 * buf, a + off, bd + off, IDESC_S, kk > 0 ? 1u : 0u);
                 }
                 mma_commit(bar(L::S_FULL + 2 * buf + sp.t));
-                if (last_use(w, sp)) mma_commit(bar(L::K_EMPTY + st));
+                if (last_use<DUAL>(w, sp)) mma_commit(bar(L::K_EMPTY + st));
               }
             } else {
-              const uint32_t vp = pos + sp.j;
+              const uint32_t vp = pos + slot;
               const uint32_t st = vp % L::V_STAGES;
-              if (sp.j > ready_j) {
+              if (slot > ready_j) {
                 if (!warp_wait(bar(L::V_FULL + st), (vp / L::V_STAGES) & 1, SITE_MMA_KV_FULL)) {
                   ok = false;
                   break;
                 }
-                ready_j = sp.j;
+                ready_j = slot;
               }
               if (!warp_wait(bar(L::P_FULL + buf), round & 1, SITE_MMA_P_FULL)) {
                 ok = false;
@@ -684,7 +729,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                          IDESC_O, (sp.j > 0 || kk > 0) ? 1u : 0u);
                 mma_commit(bar(L::O_READY + sp.t));
                 mma_commit(bar(L::PV_DONE + buf));
-                if (last_use(w, sp)) mma_commit(bar(L::V_EMPTY + st));
+                if (last_use<DUAL>(w, sp)) mma_commit(bar(L::V_EMPTY + st));
               }
             }
             ++g;
@@ -698,7 +743,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // once those MMAs complete
           if (is_s && leader) mma_commit(bar(L::Q_EMPTY));
           __syncwarp();
-          pos += w.nmax;
+          pos += DUAL ? w.nmax * w.kvs : w.nmax;
         }
       }
       // All MMAs (and their commits) must be finished before TMEM is freed.
@@ -730,7 +775,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       sync_phase ^= 1;
       return __all_sync(0xffffffffu, r);
     };
-    WorkCursor<SPLIT> cur(p);
+    WorkCursor<SPLIT, DUAL> cur(p);
     Unit w;
     while (ok && cur.next(p, w)) {
       {
@@ -738,7 +783,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t item_sk = sk;
         sk += w.n[0] + w.n[1];
         if (n == 0 && (!SPLIT || w.pieces == 1)) continue;
-        const int q_start = w.q0 + t * BLOCK_M;
+        const int q_start = (DUAL && t) ? w.q1 : w.q0 + t * BLOCK_M;
+        const int bh = (DUAL && t) ? w.bh1 : w.bh;
         const int row = q_start + r;
         // last key this row may see (top-left causal: key j <= query i)
         const int last_key = p.causal ? min(p.Nk - 1, row) : (p.Nk - 1);
@@ -872,7 +918,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           inv_self = inv_l;
           if (!SPLIT || w.pieces == 1) {
             uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
-                                                   (static_cast<size_t>(w.bh) * p.Nq + row) * D);
+                                                   (static_cast<size_t>(bh) * p.Nq + row) * D);
 #pragma unroll
             for (int c0 = 0; c0 < D; c0 += 32) {
               uint32_t o[32];
@@ -891,7 +937,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
             }
             if (p.lse != nullptr && in_range)
-              p.lse[static_cast<size_t>(w.bh) * p.Nq + row] = lse_row;
+              p.lse[static_cast<size_t>(bh) * p.Nq + row] = lse_row;
           } else {
             // a piece of a split unit: normalised O and lse to this CTA's slot
             const int slot = w.piece == 0 ? 1 : 0;
@@ -953,7 +999,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             const float w_self = ex2_approx((lse_self - lse_max) * 1.4426950408889634f);
             float wsum = 0.f;
             uint4* orow = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(p.o) +
-                                                   (static_cast<size_t>(w.bh) * p.Nq + row) * D);
+                                                   (static_cast<size_t>(bh) * p.Nq + row) * D);
             // Pieces are summed in piece order whichever CTA merges, and the
             // own piece's values are formed exactly as they were stored, so
             // the result is bit-for-bit the same on every call.
@@ -1007,7 +1053,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               }
             }
             if (p.lse != nullptr && in_range)
-              p.lse[static_cast<size_t>(w.bh) * p.Nq + row] =
+              p.lse[static_cast<size_t>(bh) * p.Nq + row] =
                   lse_max + lg2_approx(wsum) * 0.69314718055994531f;
           }
         }

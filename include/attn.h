@@ -61,16 +61,20 @@ typedef struct {
   int num_q_tiles;   /* ceil(Nq / 128): 128-row query tiles per (batch, head)            */
   int num_q_pairs;   /* ceil(num_q_tiles / 2): query tiles are processed in pairs         */
   int num_kv_tiles;  /* ceil(Nk / 128): 128-key tiles per (batch, head)                   */
-  int units_per_head; /* work units per (batch, head): num_q_pairs, or for causal
-                         ceil(num_q_pairs / 2) (a heavy query pair with its mirror)          */
-  int num_units;     /* B * H * units_per_head work units                                 */
+  int units_per_head; /* work units per (batch, head): num_q_pairs; for causal
+                         ceil(num_q_pairs / 2) (a heavy query pair with its mirror); with
+                         dual units num_q_tiles / 2 (the full query pairs)                  */
+  int num_units;     /* B * H * units_per_head + dual_units work units (unit mode)        */
+  int dual_units;    /* non-causal, odd num_q_tiles, B * H >= 2: ceil(B * H / 2) units that
+                        each pair the lone last query tile of two heads; else 0            */
   int grid;          /* persistent CTAs launched: min(num_units, SM count)                */
   int block;         /* threads per CTA                                                   */
   int smem_bytes;    /* dynamic shared memory per CTA                                     */
   int stages;        /* K/V shared-memory ring slots                                      */
   long long qk_tile_products; /* 128x128 score tiles computed (incl. masked tail tiles)   */
   int split;         /* 1 if attn_fwd_ws would use split mode for these sizes (see below)  */
-  int split_grid;    /* CTAs launched in split mode: min(SM count, units * num_kv_tiles)   */
+  int split_grid;    /* CTAs launched in split mode: min(SM count, split_units * num_kv_tiles) */
+  int split_units;   /* units split mode shares out: B * H * num_q_pairs (no dual units)  */
   long long workspace_bytes; /* workspace attn_fwd_ws needs for split mode; 0 if unused    */
 } attn_plan_t;
 

@@ -137,12 +137,22 @@ def test_plan_geometry():
     assert p["grid"] == 4 and p["block"] == 384
     assert p["qk_tile_products"] == 2 * 4 * 4
     p = A.attn_plan(16, 4, 1600, 1600, 64, 0, 148)
-    assert (p["num_q_tiles"], p["num_q_pairs"], p["num_units"], p["grid"]) == (13, 7, 448, 148)
-    # 448 units on 148 SMs leave a ragged fourth wave: split
-    assert (p["split"], p["split_grid"]) == (1, 148)
-    assert p["workspace_bytes"] == 148 * 2 * 2 * 128 * 65 * 4 + 448 * 4 + 16
+    # 13 query tiles per head: 6 full pairs per head, and the 64 lone last tiles
+    # paired across heads in 32 dual units -> 416 units, at most 3 per SM: unit mode
+    assert (p["num_q_tiles"], p["num_q_pairs"], p["units_per_head"], p["dual_units"],
+            p["num_units"], p["grid"]) == (13, 7, 6, 32, 416, 148)
+    assert p["split"] == 0 and p["workspace_bytes"] == 0
+    assert p["split_units"] == 64 * 7  # what split mode would share out (plain units)
     p3 = A.attn_plan(16, 4, 6400, 6400, 64, 0, 148)  # 1600 units: 98 % even already
-    assert p3["split"] == 0 and p3["workspace_bytes"] == 0
+    assert p3["split"] == 0 and p3["workspace_bytes"] == 0 and p3["dual_units"] == 0
+    # dual units that still leave most SMs idle: split mode over the plain units
+    p4 = A.attn_plan(1, 3, 300, 300, 64, 0, 148)
+    assert (p4["units_per_head"], p4["dual_units"], p4["num_units"]) == (1, 2, 5)
+    assert (p4["split"], p4["split_units"], p4["split_grid"]) == (1, 6, 18)
+    assert p4["workspace_bytes"] == 18 * 2 * 2 * 128 * 65 * 4 + 6 * 4 + 16
+    # no dual units for causal problems or a single head
+    assert A.attn_plan(4, 4, 300, 300, 64, 1, 148)["dual_units"] == 0
+    assert A.attn_plan(1, 1, 300, 300, 64, 0, 148)["dual_units"] == 0
     assert p["smem_bytes"] <= 232448
     p = A.attn_plan(32, 16, 2048, 2048, 64, 1, 148)
     assert p["split"] == 0  # causal work is balanced by the mirror pairing instead
