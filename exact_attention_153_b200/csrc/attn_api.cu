@@ -309,6 +309,56 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Pipelined host entry: three non-blocking streams and the events that chain
+// them, created once per device on first use (with that device current) and
+// kept for the life of the process.  One mutex per device serialises the
+// enqueue of concurrent host-entry calls on the shared streams.
+constexpr int kHostPipeMaxChunks = 8;
+constexpr size_t kHostPipeMinChunkBytes = 2u << 20;  // input bytes below which a chunk is not worth it
+
+struct HostPipe {
+  bool ready = false;
+  std::mutex mu;
+  cudaStream_t h2d = nullptr, comp = nullptr, d2h = nullptr;
+  cudaEvent_t start = nullptr, end = nullptr;
+  cudaEvent_t in_done[kHostPipeMaxChunks] = {}, comp_done[kHostPipeMaxChunks] = {};
+};
+HostPipe g_host_pipe[kMaxDevices];
+
+int host_pipe(int dev, HostPipe** out) {
+  std::lock_guard<std::mutex> lock(g_dev_mutex);
+  HostPipe& hp = g_host_pipe[dev];
+  if (!hp.ready) {
+    const unsigned int ef = cudaEventDisableTiming;
+    bool ok = cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.comp, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.start, ef) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.end, ef) == cudaSuccess;
+    for (int c = 0; ok && c < kHostPipeMaxChunks; ++c)
+      ok = cudaEventCreateWithFlags(&hp.in_done[c], ef) == cudaSuccess &&
+           cudaEventCreateWithFlags(&hp.comp_done[c], ef) == cudaSuccess;
+    if (!ok) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    hp.ready = true;
+  }
+  *out = &hp;
+  return ATTN_OK;
+}
+
+// Chunks for a problem of bh (batch, head) slices: up to kHostPipeMaxChunks,
+// each with at least kHostPipeMinChunkBytes of input.
+int host_pipe_chunks(long long bh, size_t q_head, size_t kv_head) {
+  const size_t in_bytes = static_cast<size_t>(bh) * (q_head + 2 * kv_head);
+  long long c = static_cast<long long>(in_bytes / kHostPipeMinChunkBytes);
+  if (c > kHostPipeMaxChunks) c = kHostPipeMaxChunks;
+  if (c > bh) c = bh;
+  return c < 1 ? 1 : static_cast<int>(c);
+}
+
 extern "C" {
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
@@ -354,22 +404,87 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
     return ATTN_ERR_NULL;
   int st = check_args(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Nq, Nk, d, scale, dtype);
   if (st != ATTN_OK) return st;
-  const size_t bh = static_cast<size_t>(B) * H;
-  const size_t q_bytes = bh * Nq * d * 2, kv_bytes = bh * Nk * d * 2;
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(q_dev, q_host, q_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(k_dev, k_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-      cudaMemcpyAsync(v_dev, v_host, kv_bytes, cudaMemcpyHostToDevice, s) != cudaSuccess) {
-    cudaGetLastError();
-    return ATTN_ERR_CUDA;
-  }
-  st = fwd_impl(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Nq, Nk, d, scale, causal, dtype,
-                workspace, workspace_bytes, stream);
+  int dev = -1;
+  DeviceInfo* info = nullptr;
+  st = current_device(&dev, &info);
   if (st != ATTN_OK) return st;
-  if (cudaMemcpyAsync(o_host, o_dev, q_bytes, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-      (lse_host != nullptr && lse_dev != nullptr &&
-       cudaMemcpyAsync(lse_host, lse_dev, bh * Nq * sizeof(float), cudaMemcpyDeviceToHost, s) !=
-           cudaSuccess)) {
+  const long long bh = static_cast<long long>(B) * H;
+  const size_t q_head = static_cast<size_t>(Nq) * d * 2, kv_head = static_cast<size_t>(Nk) * d * 2;
+  const bool with_lse = lse_host != nullptr && lse_dev != nullptr;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+
+  attn_plan_t plan;
+  fill_plan(B, H, Nq, Nk, d, causal, info->sms, &plan);
+  const bool uses_split = plan.split && workspace != nullptr &&
+                          workspace_bytes >= static_cast<size_t>(plan.workspace_bytes);
+  const int chunks = host_pipe_chunks(bh, q_head, kv_head);
+  if (uses_split || chunks < 2) {
+    // one shot on the caller's stream: copies in, forward, copies out
+    if (cudaMemcpyAsync(q_dev, q_host, bh * q_head, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(k_dev, k_host, bh * kv_head, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(v_dev, v_host, bh * kv_head, cudaMemcpyHostToDevice, s) != cudaSuccess) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    st = fwd_impl(q_dev, k_dev, v_dev, o_dev, lse_dev, B, H, Nq, Nk, d, scale, causal, dtype,
+                  workspace, workspace_bytes, stream);
+    if (st != ATTN_OK) return st;
+    if (cudaMemcpyAsync(o_host, o_dev, bh * q_head, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        (with_lse && cudaMemcpyAsync(lse_host, lse_dev, bh * Nq * sizeof(float),
+                                     cudaMemcpyDeviceToHost, s) != cudaSuccess)) {
+      cudaGetLastError();
+      return ATTN_ERR_CUDA;
+    }
+    return ATTN_OK;
+  }
+
+  // Pipelined over chunks of consecutive (batch, head) slices, which are
+  // contiguous in every tensor: chunk c's host->device copies, its forward
+  // and its device->host copies run on three library streams, so the copies
+  // of one chunk overlap the compute and the opposite-direction copies of
+  // the others.  Unit mode computes every row the same way whichever unit
+  // holds it, so the result is bit-for-bit that of attn_fwd.
+  HostPipe* hp = nullptr;
+  st = host_pipe(dev, &hp);
+  if (st != ATTN_OK) return st;
+  std::lock_guard<std::mutex> lock(hp->mu);
+  const long long per = (bh + chunks - 1) / chunks;
+  bool ok = cudaEventRecord(hp->start, s) == cudaSuccess &&
+            cudaStreamWaitEvent(hp->h2d, hp->start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(hp->comp, hp->start, 0) == cudaSuccess &&
+            cudaStreamWaitEvent(hp->d2h, hp->start, 0) == cudaSuccess;
+  for (int c = 0; ok && c < chunks; ++c) {
+    const long long h0 = c * per;
+    const long long nh = (h0 + per <= bh) ? per : bh - h0;
+    if (nh <= 0) break;
+    const size_t qo = static_cast<size_t>(h0) * q_head, kvo = static_cast<size_t>(h0) * kv_head;
+    const size_t lo = static_cast<size_t>(h0) * Nq;
+    ok = cudaMemcpyAsync(static_cast<char*>(q_dev) + qo, static_cast<const char*>(q_host) + qo,
+                         nh * q_head, cudaMemcpyHostToDevice, hp->h2d) == cudaSuccess &&
+         cudaMemcpyAsync(static_cast<char*>(k_dev) + kvo, static_cast<const char*>(k_host) + kvo,
+                         nh * kv_head, cudaMemcpyHostToDevice, hp->h2d) == cudaSuccess &&
+         cudaMemcpyAsync(static_cast<char*>(v_dev) + kvo, static_cast<const char*>(v_host) + kvo,
+                         nh * kv_head, cudaMemcpyHostToDevice, hp->h2d) == cudaSuccess &&
+         cudaEventRecord(hp->in_done[c], hp->h2d) == cudaSuccess &&
+         cudaStreamWaitEvent(hp->comp, hp->in_done[c], 0) == cudaSuccess;
+    if (!ok) break;
+    st = fwd_impl(static_cast<char*>(q_dev) + qo, static_cast<char*>(k_dev) + kvo,
+                  static_cast<char*>(v_dev) + kvo, static_cast<char*>(o_dev) + qo,
+                  lse_dev != nullptr ? lse_dev + lo : nullptr, static_cast<int>(nh), 1, Nq, Nk, d,
+                  scale, causal, dtype, nullptr, 0, reinterpret_cast<attn_stream_t>(hp->comp));
+    if (st != ATTN_OK) return st;
+    ok = cudaEventRecord(hp->comp_done[c], hp->comp) == cudaSuccess &&
+         cudaStreamWaitEvent(hp->d2h, hp->comp_done[c], 0) == cudaSuccess &&
+         cudaMemcpyAsync(static_cast<char*>(o_host) + qo, static_cast<char*>(o_dev) + qo,
+                         nh * q_head, cudaMemcpyDeviceToHost, hp->d2h) == cudaSuccess &&
+         (!with_lse || cudaMemcpyAsync(lse_host + lo, lse_dev + lo, nh * Nq * sizeof(float),
+                                       cudaMemcpyDeviceToHost, hp->d2h) == cudaSuccess);
+  }
+  // the caller's stream continues after the last copy back (which itself
+  // followed every chunk's forward and copies in)
+  ok = ok && cudaEventRecord(hp->end, hp->d2h) == cudaSuccess &&
+       cudaStreamWaitEvent(s, hp->end, 0) == cudaSuccess;
+  if (!ok) {
     cudaGetLastError();
     return ATTN_ERR_CUDA;
   }

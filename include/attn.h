@@ -189,14 +189,26 @@ int attn_fwd_stall_test(const void* q, const void* k, const void* v, void* o, fl
 /*
  * attn_fwd_host -- the same forward, end to end from host memory.
  *
- * Enqueues on `stream`: host->device copies of q_host, k_host, v_host into the caller's
- * device buffers q_dev, k_dev, v_dev; attn_fwd on them into o_dev / lse_dev; device->host
- * copies of o_dev into o_host and (when both lse pointers are non-NULL) lse_dev into
- * lse_host.  Host buffers should be pinned (cudaHostAlloc / cudaHostRegister) for the copies
- * to be asynchronous.  The caller synchronises `stream` before reading o_host.  Argument
- * rules and error codes are those of attn_fwd; every host and device pointer except the lse
- * pair must be non-NULL.  workspace / workspace_bytes are optional (NULL, 0) and act as in
- * attn_fwd_ws.  Nothing is allocated.
+ * Host->device copies of q_host, k_host, v_host into the caller's device buffers q_dev,
+ * k_dev, v_dev; the forward on them into o_dev / lse_dev; device->host copies of o_dev into
+ * o_host and (when both lse pointers are non-NULL) lse_dev into lse_host.  The whole call is
+ * ordered after the work already enqueued on `stream`, and work enqueued on `stream`
+ * afterwards runs after it; the caller synchronises `stream` before reading o_host.  Host
+ * buffers must be pinned (cudaHostAlloc / cudaHostRegister) for the copies to be
+ * asynchronous.
+ *
+ * Problems with at least 4 MB of input that run in unit mode are pipelined: the (batch,
+ * head) slices are cut into up to 8 contiguous chunks, and chunk c's copies in, forward and
+ * copies out run on three streams the library creates once per device (with events chaining
+ * them), so copies of one chunk overlap the compute and the opposite-direction copies of
+ * the others.  The result is bit-for-bit that of attn_fwd.  Calls from several host threads
+ * share those streams and are serialised by a lock while they enqueue.  Smaller problems,
+ * and problems that take split mode from `workspace`, run as one copy-in / forward /
+ * copy-out sequence on `stream`.
+ *
+ * Argument rules and error codes are those of attn_fwd; every host and device pointer
+ * except the lse pair must be non-NULL.  workspace / workspace_bytes are optional (NULL, 0)
+ * and act as in attn_fwd_ws.  Nothing is allocated per call.
  */
 int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
                   float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,

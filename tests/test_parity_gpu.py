@@ -356,3 +356,36 @@ def test_yolo_40x40_uses_dual_units_not_split():
     p = A.attn_plan(w.B, w.H, w.Nq, w.Nk, w.d, int(w.causal),
                     torch.cuda.get_device_properties(0).multi_processor_count)
     assert p["dual_units"] == 32 and p["num_units"] == 416 and p["split"] == 0
+
+
+# ------------------------------------------------------------ pipelined host entry
+
+@pytest.mark.parametrize("B,H,N,d,dtype,causal,with_lse", [
+    (4, 8, 2048, 64, "fp16", True, True),     # 25 MB in: 8 chunks of 4 heads
+    (1, 13, 1000, 128, "bf16", False, False),  # 13 heads: 7 chunks, the last with one head
+    (16, 4, 1600, 64, "fp16", False, True),   # the 40x40 YOLO shape (dual units per chunk)
+])
+def test_host_entry_pipelined_matches_device_entry(B, H, N, d, dtype, causal, with_lse):
+    """Chunked copies and forwards on library streams give the bits of attn_fwd, ordered on the
+    caller's stream: earlier work on it finishes first, later work sees the results."""
+    q, k, v = make_qkv(B, H, N, N, d, dtype, seed=B * H + N + d)
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((B, H, N), dtype=torch.float32).pin_memory() if with_lse else None
+    qd, kd, vd = (torch.empty_like(t, device="cuda") for t in (q, k, v))
+    od = torch.empty_like(qd)
+    ld = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        od.fill_(7.0)  # earlier work on the caller's stream
+        torch.cuda._sleep(1_000_000)
+        A.forward_host(qh, kh, vh, oh, lh, qd, kd, vd, od, ld, causal=causal, stream=side)
+        o_after = od.clone()  # later work on the caller's stream
+    side.synchronize()
+    o, lse = A.forward(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    torch.cuda.synchronize()
+    assert torch.equal(oh, o.cpu())
+    assert torch.equal(o_after, o)
+    if with_lse:
+        assert torch.equal(lh, lse.cpu())
+    assert A.attn_get_device_status()[0] == 0
