@@ -76,7 +76,7 @@ def recorded_traffic(workload: str):
     with open(TRAFFIC_FILE) as f:
         doc = json.load(f)
     ent = doc.get("workloads", {}).get(workload)
-    if not ent or ent.get("kernel_source_sha") != kernel_source_sha():
+    if not ent or doc.get("kernel_source_sha") != kernel_source_sha():
         return None
     return ent.get("dram_bytes_per_launch")
 

@@ -1,0 +1,39 @@
+"""bench.py host logic on the CPU: the roofline arithmetic and the recorded-traffic lookup."""
+import json
+
+import bench
+from seeded_inputs import workload
+
+PEAKS = {"bf16_tflops": 1653.3, "bf16_tflops_sustained": 1396.4, "hbm_gbs": 6544.0}
+
+
+def test_roofline_tensor_bound():
+    w = workload("yolo_highres_80x80_b16")
+    t = w.flops / 800e12  # a launch that reaches 800 TFLOP/s
+    r = bench.roofline(w, t, PEAKS)
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert abs(r["achieved"] - 800.0) < 0.01 and abs(r["frac"] - 800.0 / 1653.3) < 1e-4
+    rs = bench.roofline(w, t, PEAKS, sustained=True)
+    assert abs(rs["frac"] - 800.0 / 1396.4) < 1e-4
+
+
+def test_roofline_hbm_bound_below_the_ridge_point():
+    w = workload("yolo_c2psa_20x20")  # 200 FLOP per byte, ridge point 253
+    assert w.flops / w.bytes < 1653.3e12 / 6544e9
+    t = w.bytes / 1000e9
+    r = bench.roofline(w, t, PEAKS)
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert abs(r["achieved"] - 1000.0) < 0.1
+
+
+def test_recorded_traffic_only_for_current_sources(tmp_path, monkeypatch):
+    path = tmp_path / "traffic.json"
+    doc = {"kernel": "k", "kernel_source_sha": bench.kernel_source_sha(),
+           "workloads": {"yolo_neck_40x40_b16": {"dram_bytes_per_launch": 123.0}}}
+    path.write_text(json.dumps(doc))
+    monkeypatch.setattr(bench, "TRAFFIC_FILE", str(path))
+    assert bench.recorded_traffic("yolo_neck_40x40_b16") == 123.0
+    assert bench.recorded_traffic("long_context_32k") is None
+    doc["kernel_source_sha"] = "0" * 16  # counters taken on other sources
+    path.write_text(json.dumps(doc))
+    assert bench.recorded_traffic("yolo_neck_40x40_b16") is None
