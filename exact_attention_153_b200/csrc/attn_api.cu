@@ -81,16 +81,25 @@ int check_args(const void* q, const void* k, const void* v, const void* o, const
   return ATTN_OK;
 }
 
-// Split mode pays off when whole units would leave a ragged last wave: the
-// CTAs that run one unit more set the kernel time.  It needs a workspace and
-// is used for non-causal problems whose unit count spreads over the grid
-// with less than 90 % efficiency.
-bool split_pays(long long units, long long total_steps, int num_sms, int causal) {
+// Split mode pays when unit mode leaves the grid ragged (fewer units than
+// SMs, or a last wave under 90 % full) and the serial key-tile steps it saves
+// per CTA outweigh its own cost: publishing and merging the pieces of a unit
+// (the last piece reads every other piece's O back).  The cost, in key-tile
+// steps, was fitted to split and unit timings of small problems on B200:
+// about 3.5 + 0.56 per piece at d = 64 and 2.5 + 1.03 per piece at d = 128.
+bool split_pays(long long units, int kv_tiles, long long total_steps, int num_sms, int causal,
+                int d) {
   if (causal || total_steps < 2) return false;
   const long long grid = units < num_sms ? units : num_sms;
   const long long waves = (units + grid - 1) / grid;
   const double eff = static_cast<double>(units) / static_cast<double>(grid * waves);
-  return eff < 0.9 || units < num_sms;
+  if (eff >= 0.9 && units >= num_sms) return false;
+  const long long steps_unit = waves * kv_tiles;
+  const long long grid_s = total_steps < num_sms ? total_steps : num_sms;
+  const long long steps_split = (total_steps + grid_s - 1) / grid_s;
+  const long long pieces = (static_cast<long long>(kv_tiles) * grid_s + total_steps - 1) / total_steps;
+  const double cost = d == 64 ? 3.5 + 0.56 * pieces : 2.5 + 1.03 * pieces;
+  return static_cast<double>(steps_unit - steps_split) > cost;
 }
 
 size_t split_workspace_bytes(int grid, int d, long long units) {
@@ -135,7 +144,7 @@ void fill_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, att
   // split mode keeps plain units (one (batch, head) each): q_pairs per head
   const long long split_units = BH * q_pairs;
   const long long total_steps = split_units * kv_tiles;
-  out->split = (!causal && split_pays(units, total_steps, num_sms, causal)) ? 1 : 0;
+  out->split = split_pays(units, kv_tiles, total_steps, num_sms, causal, d) ? 1 : 0;
   out->split_grid = static_cast<int>(total_steps < num_sms ? total_steps : num_sms);
   out->split_units = static_cast<int>(split_units);
   out->workspace_bytes =

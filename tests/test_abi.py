@@ -132,8 +132,16 @@ def test_workspace_entry_argument_errors():
 def test_plan_geometry():
     p = A.attn_plan(1, 2, 400, 400, 64, 0, 148)
     assert (p["num_q_tiles"], p["num_q_pairs"], p["num_kv_tiles"], p["num_units"]) == (4, 2, 4, 4)
-    # fewer units than SMs: split mode spreads the 4 x 4 (unit, key tile) steps over 16 CTAs
-    assert (p["split"], p["split_grid"]) == (1, 16) and p["workspace_bytes"] > 0
+    # 4 units of 4 key tiles: splitting saves 3 serial steps, less than it costs to merge
+    # 4 pieces per unit, so unit mode
+    assert p["split"] == 0 and p["workspace_bytes"] == 0 and p["split_grid"] == 16
+    ps = A.attn_plan(1, 1, 2000, 2000, 64, 0, 148)
+    # 8 units of 16 key tiles: 16 serial steps per CTA against 1 step and 16-piece merges
+    assert (ps["split"], ps["split_grid"], ps["split_units"]) == (1, 128, 8)
+    assert ps["workspace_bytes"] == 128 * 2 * 2 * 128 * 65 * 4 + 8 * 4 + 16
+    assert A.attn_plan(1, 4, 1000, 1000, 64, 0, 148)["split"] == 0  # 7 steps saved, 8 pieces
+    pd = A.attn_plan(2, 2, 512, 8192, 128, 0, 148)  # d = 128: 64 steps against 4 + 19 pieces
+    assert (pd["split"], pd["split_grid"]) == (1, 148)
     assert p["grid"] == 4 and p["block"] == 384
     assert p["qk_tile_products"] == 2 * 4 * 4
     p = A.attn_plan(16, 4, 1600, 1600, 64, 0, 148)
@@ -145,11 +153,14 @@ def test_plan_geometry():
     assert p["split_units"] == 64 * 7  # what split mode would share out (plain units)
     p3 = A.attn_plan(16, 4, 6400, 6400, 64, 0, 148)  # 1600 units: 98 % even already
     assert p3["split"] == 0 and p3["workspace_bytes"] == 0 and p3["dual_units"] == 0
-    # dual units that still leave most SMs idle: split mode over the plain units
     p4 = A.attn_plan(1, 3, 300, 300, 64, 0, 148)
     assert (p4["units_per_head"], p4["dual_units"], p4["num_units"]) == (1, 2, 5)
-    assert (p4["split"], p4["split_units"], p4["split_grid"]) == (1, 6, 18)
-    assert p4["workspace_bytes"] == 18 * 2 * 2 * 128 * 65 * 4 + 6 * 4 + 16
+    assert (p4["split"], p4["split_units"], p4["split_grid"]) == (0, 6, 18)
+    # dual units in unit mode, but split mode (over the plain units) when it pays
+    p5 = A.attn_plan(1, 2, 300, 4000, 64, 0, 148)
+    assert (p5["dual_units"], p5["num_units"], p5["split_units"]) == (1, 3, 4)
+    assert (p5["split"], p5["split_grid"]) == (1, 128)
+    assert p5["workspace_bytes"] == 128 * 2 * 2 * 128 * 65 * 4 + 4 * 4 + 16
     # no dual units for causal problems or a single head
     assert A.attn_plan(4, 4, 300, 300, 64, 1, 148)["dual_units"] == 0
     assert A.attn_plan(1, 1, 300, 300, 64, 0, 148)["dual_units"] == 0

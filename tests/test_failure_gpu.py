@@ -43,8 +43,11 @@ CASES = [
 def test_injected_stall_times_out_and_context_recovers(site, split, d):
     dtype = "fp16" if d == 64 else "bf16"
     code = A.ATTN_FP16 if d == 64 else A.ATTN_BF16
-    B, H, N = 1, 2, (400 if split else 300)
-    Nk = N if d == 64 else 1700  # d = 128 split needs several pieces per unit
+    if split:  # shapes for which attn_fwd_ws takes split mode
+        B, H, N, Nk = (1, 1, 2000, 2000) if d == 64 else (2, 2, 512, 8192)
+    else:
+        B, H, N = 1, 2, 300
+        Nk = N if d == 64 else 1700
     q, k, v = make_qkv(B, H, N, Nk, d, dtype, seed=site * 10 + d)
     qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
     o = torch.empty_like(qd)
