@@ -11,21 +11,28 @@
 // tile at a time.
 //
 // Blackwell mapping (one CTA per SM, persistent over work units):
-//   * a work unit is two 128-row Q tiles of one (batch, head); the two tiles
-//     share every K/V tile the CTA loads;
-//   * warp 9 (one lane) issues TMA loads: the unit's two Q tiles, then K_j and
-//     V_j for j = 0..n-1 into a ring of STAGES shared-memory slots, each slot
-//     guarded by a full / empty mbarrier pair;
-//   * warp 8 (one lane) issues tcgen05.mma: S_t = Q_t K_j^T into TMEM (fp32),
-//     and O_t += P_t V_j with P_t read from TMEM (it overwrites S_t, packed
-//     as 16-bit pairs); tcgen05.commit signals the softmax warps and releases
-//     ring slots;
-//   * warps 0-3 own Q tile 0 and warps 4-7 own Q tile 1: one thread per
-//     query row reads its S row from TMEM, masks, updates the running max
-//     m (base-2, pre-multiplied by scale*log2 e) and sum l, writes P, and
-//     rescales its O row in TMEM by 2^(m_old - m_new) when the max rose.
-//     While one warpgroup runs its softmax the tensor core works on the
-//     other tile, so exp and MMA overlap.
+//   * a work unit is two 128-row Q tiles of one (batch, head) that share
+//     every K/V tile the CTA loads (a dual unit: the last tiles of two heads,
+//     each with its own K/V stream); causal units pair a heavy query pair
+//     with its light mirror; split mode shares a ragged grid's key-tile steps
+//     out evenly and merges the pieces in the log domain;
+//   * warp 9 issues the TMA loads of the unit's Q tiles and of K_j into a
+//     ring of K slots, warp 11 those of V_j into a ring of V slots, each slot
+//     guarded by a full / empty mbarrier pair (128-byte swizzle, no
+//     multicast);
+//   * warp 8 issues tcgen05.mma S = Q_t K_j^T (fp32) into one of NSB TMEM S/P
+//     buffers as soon as K_j is in and the buffer's last P V is done, so it
+//     runs ahead of the softmax; warp 10 issues O_t += P V_j with P read from
+//     TMEM, where the softmax wrote it over S as 16-bit pairs (at d = 128,
+//     with two buffers, warp 8 issues both in sequence order).  The producer
+//     warps loop on all lanes and one elected lane issues; tcgen05.commit
+//     signals the softmax warps and releases ring slots;
+//   * warps 0-3 own Q tile 0 and warps 4-7 Q tile 1, one thread per query
+//     row: each reads its S row from TMEM, masks, keeps the running max m
+//     (base 2, pre-multiplied by scale * log2 e) and sum l, writes P, and
+//     rescales its O row in TMEM by 2^(m_old - m_new) when the max rose by
+//     more than the lazy threshold.  While one warpgroup runs its softmax the
+//     tensor core works on the other tile, so exponentials and MMAs overlap;
 //   * the epilogue divides O by l, rounds to the input dtype and stores the
 //     rows below Nq; lse = (m + log2 l) * ln 2.
 //

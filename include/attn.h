@@ -173,7 +173,8 @@ int attn_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float
  *   stall_site 1: softmax warpgroup 0, before its first score tile;
  *              2: the MMA warp, before its first MMA;
  *              3: the Q/K TMA warp, before its first load;
- *              4: softmax warpgroup 0, before the split-piece rendezvous (split mode only).
+ *              4: softmax warpgroup 0, before the split-piece rendezvous (split mode only;
+ *                 the shapes for which attn_plan reports split = 1).
  * The kernel records 0x8000000A in the device status word, every role leaves its loop, the
  * issued loads and MMAs are waited for, tensor memory is freed and the kernel returns;
  * attn_get_device_status() then reports ATTN_ERR_DEVICE_TIMEOUT and the CUDA context stays
