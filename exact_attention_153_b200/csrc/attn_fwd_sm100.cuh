@@ -396,6 +396,35 @@ __device__ __forceinline__ bool last_use(const Unit& w, SeqPos s) {
   return (DUAL && w.kvs == 2) || s.t == 1 || s.j >= w.n[1];
 }
 
+// P for one 128-key row: p = 2^(s * sl2 + neg_m), packed two keys per word
+// (even key low), and the fp32 sum of the unrounded values.  Of every 16 key
+// pairs, exp_poly_pairs<D>() take 2^x from the FMA-pipe polynomial.
+// d = 64 (bound by the softmax) tries the running max as it stands before
+// computing a row max; at d = 128 the extra registers of that path cost more
+// than it saves.
+template <int D>
+__host__ __device__ constexpr bool kStaleMaxFirst() { return D == 64; }
+
+template <int D, bool BF16>
+__device__ __forceinline__ float exp_row(const float (&s)[128], float sl2, float neg_m,
+                                         uint32_t (&pk)[64]) {
+  float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+  for (int i = 0; i < 64; ++i) {
+    float x0, x1, a, bb;
+    fma2(x0, x1, s[2 * i], s[2 * i + 1], sl2, sl2, neg_m, neg_m);
+    if (i % 16 < exp_poly_pairs<D>()) {
+      exp2_poly2(a, bb, x0, x1);  // FMA pipe, in parallel with the MUFU ones
+    } else {
+      a = ex2_approx(x0);
+      bb = ex2_approx(x1);
+    }
+    add2(sum0, sum1, sum0, sum1, a, bb);
+    pk[i] = pack2<BF16>(a, bb);
+  }
+  return sum0 + sum1;
+}
+
 // Bounded wait on one mbarrier phase, fully inlined (a call here would make
 // the compiler save live registers to local memory on every slow wait).
 // Returns false on timeout (status word set, abort flag raised) or, when
@@ -811,70 +840,140 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!ok) break;
           s_parity ^= 1u << b;
           tc_fence_after();
-          uint32_t sr[128];
+          bool raise = false;
+          float alpha = 1.f, m_new = m;
+          if constexpr (kStaleMaxFirst<D>()) {
+            // S of this tile, keys past the row's last visible key set to -inf
+            float s[128];
+            auto load_s = [&]() {
+              uint32_t sr[128];
 #pragma unroll
-          for (int c = 0; c < 4; ++c)
-            tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * c));
-          tmem_wait_ld_regs(sr);
-          float s[128];
+              for (int c = 0; c < 4; ++c)
+                tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * c));
+              tmem_wait_ld_regs(sr);
 #pragma unroll
-          for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
-
-          const int k0 = (w.jbase + j) * BLOCK_N;
-          const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > q_start);
-          if (need_mask) {
-            const int lim = last_key - k0;  // columns > lim are masked
+              for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+              const int k0 = (w.jbase + j) * BLOCK_N;
+              const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > q_start);
+              if (need_mask) {
+                const int lim = last_key - k0;  // columns > lim are masked
 #pragma unroll
-            for (int c = 0; c < 128; ++c) s[c] = (c > lim) ? -INFINITY : s[c];
-          }
-          // row max: eight independent chains of three-input max over s[0..127]
-          float mx[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) mx[i] = max3(s[2 * i], s[2 * i + 1], s[16 + 2 * i]);
-#pragma unroll
-          for (int c = 32; c < 128; c += 16) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], s[c + 2 * i], s[c + 2 * i + 1]);
-          }
-#pragma unroll
-          for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[17 + 2 * i]);
-          const float mx_all = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]),
-                                    fmaxf(mx[6], mx[7]));
-          // The running max only moves when the tile raises it by more than
-          // RESCALE_LOG2 (base 2): until then exponents stay below
-          // 2^RESCALE_LOG2 and O, l and lse keep using the same stale max, so
-          // the result is unchanged while most O rescales are skipped.
-          const float m_cand = fmaxf(m, mx_all * sl2);
-          const bool raise = m_cand > m + RESCALE_LOG2;
-          const float m_new = raise ? m_cand : m;
-          const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-          const float alpha = raise ? ex2_approx(m - m_use) : 1.f;
-          const float neg_m = -m_use;
-
-          // P = 2^(s * scale * log2 e - m), packed two keys per 32-bit TMEM
-          // column (even key in the low half), written over S in 16-column
-          // chunks so each chunk's S registers die as it is stored.
-          float sum0 = 0.f, sum1 = 0.f;
-#pragma unroll
-          for (int chunk = 0; chunk < 4; ++chunk) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              float x0, x1, a, bb;
-              fma2(x0, x1, s[32 * chunk + 2 * c], s[32 * chunk + 2 * c + 1], sl2, sl2, neg_m, neg_m);
-              if (c < exp_poly_pairs<D>()) {
-                exp2_poly2(a, bb, x0, x1);  // FMA pipe, in parallel with the MUFU ones
-              } else {
-                a = ex2_approx(x0);
-                bb = ex2_approx(x1);
+                for (int c = 0; c < 128; ++c) s[c] = (c > lim) ? -INFINITY : s[c];
               }
-              add2(sum0, sum1, sum0, sum1, a, bb);
-              pk[c] = pack2<BF16>(a, bb);
+            };
+            load_s();
+
+            // P = 2^(s * scale * log2 e - m), packed two keys per 32-bit word
+            // (even key in the low half).  After the first tile the running
+            // max m is tried as it stands: the sum of the tile's P bounds every
+            // P, so if it stays below 2^15 no P overflows a 16-bit float and
+            // the result is exact with the stale max, and the row max is
+            // never computed.  Otherwise (or on the first tile) S is read
+            // again and the row max decides, as below.  P is written to TMEM
+            // only after that decision, so S is still there to be read again.
+            uint32_t pk[64];
+            float tsum = 0.f;
+            bool settled = false;
+            if (j > 0) {
+              tsum = exp_row<D, BF16>(s, sl2, -m, pk);
+              settled = __all_sync(0xffffffffu, tsum < 32768.f);
+              if (!settled) load_s();
             }
-            tmem_st16(tS + 16 * chunk, pk);
+            if (!settled) {
+              // row max: eight independent chains of three-input max over s[0..127]
+              float mx[8];
+#pragma unroll
+              for (int i = 0; i < 8; ++i) mx[i] = max3(s[2 * i], s[2 * i + 1], s[16 + 2 * i]);
+#pragma unroll
+              for (int c = 32; c < 128; c += 16) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], s[c + 2 * i], s[c + 2 * i + 1]);
+              }
+#pragma unroll
+              for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[17 + 2 * i]);
+              const float mx_all = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]),
+                                        fmaxf(mx[6], mx[7]));
+              // The running max only moves when the tile raises it by more than
+              // RESCALE_LOG2 (base 2): until then exponents stay below
+              // 2^RESCALE_LOG2 and O, l and lse keep using the same stale max,
+              // so the result is unchanged while most O rescales are skipped.
+              const float m_cand = fmaxf(m, mx_all * sl2);
+              raise = m_cand > m + RESCALE_LOG2;
+              m_new = raise ? m_cand : m;
+              const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+              alpha = raise ? ex2_approx(m - m_use) : 1.f;
+              tsum = exp_row<D, BF16>(s, sl2, -m_use, pk);
+            }
+            tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
+            tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+            l = l * alpha + tsum;
+            m = m_new;
+          } else {
+            uint32_t sr[128];
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              tmem_ld32(tS + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(sr + 32 * c));
+            tmem_wait_ld_regs(sr);
+            float s[128];
+#pragma unroll
+            for (int c = 0; c < 128; ++c) s[c] = __uint_as_float(sr[c]);
+
+            const int k0 = (w.jbase + j) * BLOCK_N;
+            const bool need_mask = (k0 + BLOCK_N > p.Nk) || (p.causal && k0 + BLOCK_N - 1 > q_start);
+            if (need_mask) {
+              const int lim = last_key - k0;  // columns > lim are masked
+#pragma unroll
+              for (int c = 0; c < 128; ++c) s[c] = (c > lim) ? -INFINITY : s[c];
+            }
+            // row max: eight independent chains of three-input max over s[0..127]
+            float mx[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx[i] = max3(s[2 * i], s[2 * i + 1], s[16 + 2 * i]);
+#pragma unroll
+            for (int c = 32; c < 128; c += 16) {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) mx[i] = max3(mx[i], s[c + 2 * i], s[c + 2 * i + 1]);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[17 + 2 * i]);
+            const float mx_all = max3(max3(mx[0], mx[1], mx[2]), max3(mx[3], mx[4], mx[5]),
+                                      fmaxf(mx[6], mx[7]));
+            // The running max only moves when the tile raises it by more than
+            // RESCALE_LOG2 (base 2): until then exponents stay below
+            // 2^RESCALE_LOG2 and O, l and lse keep using the same stale max, so
+            // the result is unchanged while most O rescales are skipped.
+            const float m_cand = fmaxf(m, mx_all * sl2);
+            raise = m_cand > m + RESCALE_LOG2;
+            m_new = raise ? m_cand : m;
+            const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+            alpha = raise ? ex2_approx(m - m_use) : 1.f;
+            const float neg_m = -m_use;
+
+            // P = 2^(s * scale * log2 e - m), packed two keys per 32-bit TMEM
+            // column (even key in the low half), written over S in 16-column
+            // chunks so each chunk's S registers die as it is stored.
+            float sum0 = 0.f, sum1 = 0.f;
+#pragma unroll
+            for (int chunk = 0; chunk < 4; ++chunk) {
+              uint32_t pk[16];
+#pragma unroll
+              for (int c = 0; c < 16; ++c) {
+                float x0, x1, a, bb;
+                fma2(x0, x1, s[32 * chunk + 2 * c], s[32 * chunk + 2 * c + 1], sl2, sl2, neg_m, neg_m);
+                if (c < exp_poly_pairs<D>()) {
+                  exp2_poly2(a, bb, x0, x1);  // FMA pipe, in parallel with the MUFU ones
+                } else {
+                  a = ex2_approx(x0);
+                  bb = ex2_approx(x1);
+                }
+                add2(sum0, sum1, sum0, sum1, a, bb);
+                pk[c] = pack2<BF16>(a, bb);
+              }
+              tmem_st16(tS + 16 * chunk, pk);
+            }
+            l = l * alpha + (sum0 + sum1);
+            m = m_new;
           }
-          l = l * alpha + (sum0 + sum1);
-          m = m_new;
 
           // O_t may only be touched once the previous P V of this tile is
           // done: with split issue that is its own signal; with in-order issue

@@ -179,6 +179,22 @@ def test_dominant_key():
     assert _err(o[0, 0, i].double().numpy(), v[0, 0, j].double().numpy()) <= TOL["fp16"]
 
 
+@pytest.mark.parametrize("dtype", ["fp16", "bf16"])
+def test_late_keys_raise_the_running_max(dtype):
+    """Keys in later tiles whose scores exceed every earlier score by 12, 20 and 40 (base 2):
+    12 stays on the stale-max path (P up to 2^12), 20 and 40 force the row max and a raise."""
+    q, k, v = make_qkv(1, 2, 600, 900, 64, dtype, seed=26)
+    scale = 0.125
+    log2e = 1.4426950408889634
+    for n, (row, key, gap) in enumerate([(5, 300, 12.0), (130, 520, 20.0), (257, 777, 40.0),
+                                         (400, 899, 20.0), (599, 640, 12.0)]):
+        qi = q[0, n % 2, row].double()
+        # score of (row, key) = scale * |q_row| * a, in base 2: gap above the row's other scores
+        a = (gap / log2e + 4.0) / (scale * float(qi.norm()))
+        k[0, n % 2, key] = (a * qi / qi.norm()).to(k.dtype)
+    _check_full(q, k, v, False, scale, dtype)
+
+
 # ------------------------------------------------------------ memory safety, determinism
 
 @pytest.mark.parametrize("Nq,d,dtype", [(400, 64, "fp16"), (129, 128, "bf16"), (1, 64, "bf16")])
