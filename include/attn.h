@@ -107,8 +107,10 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
  * attn_fwd_ws -- attn_fwd with a caller-provided device workspace that enables split mode.
  *
  * For non-causal problems whose work units would fill the GPU unevenly (a ragged last wave,
- * or fewer units than SMs -- e.g. the 20x20 and 40x40 YOLO workloads), the kernel divides
- * the flattened (unit, key tile) range evenly over the CTAs.  A unit cut by a range boundary
+ * or fewer units than SMs) and where the serial key-tile steps this saves outweigh the cost
+ * of merging pieces (few units with many key tiles each, e.g. B = H = 1, N = 2000; attn_plan
+ * reports the decision), the kernel divides the flattened (unit, key tile) range evenly over
+ * the CTAs.  A unit cut by a range boundary
  * is computed in pieces; each piece writes its normalised O and its logsumexp to the
  * workspace and the last piece to finish merges them exactly with the log-domain identity
  * lse = ln sum_k exp(lse_k), O = sum_k exp(lse_k - lse) O_k (the saved-statistics
