@@ -18,8 +18,8 @@
 //     out evenly and merges the pieces in the log domain;
 //   * warp 9 issues the TMA loads of the unit's Q tiles and of K_j into a
 //     ring of K slots, warp 11 those of V_j into a ring of V slots, each slot
-//     guarded by a full / empty mbarrier pair (128-byte swizzle, no
-//     multicast);
+//     guarded by a full / empty mbarrier pair (128-byte swizzle; every CTA
+//     loads its own tiles);
 //   * warp 8 issues tcgen05.mma S = Q_t K_j^T (fp32) into one of NSB TMEM S/P
 //     buffers as soon as K_j is in and the buffer's last P V is done, so it
 //     runs ahead of the softmax; warp 10 issues O_t += P V_j with P read from
