@@ -1,4 +1,4 @@
-"""CPU float64 oracle for the exact attention forward.
+"""CPU float64 oracle for the exact attention forward and its gradients.
 
 TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
 and the CPU-baseline leg of ``bench.py``.  The CUDA path never imports it.
@@ -7,4 +7,8 @@ from .attention import (  # noqa: F401
     apply_causal_mask, attention_f64, attention_head_rows, attention_probs_f64,
     brute_force, logsumexp_rows, online_softmax_f64, scores, softmax_rows,
     to_f64, weighted_sum,
+)
+from .backward import (  # noqa: F401
+    attention_backward_f64, grad_k, grad_p, grad_q, grad_scores, grad_v, recompute_probs,
+    row_dot,
 )

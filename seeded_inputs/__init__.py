@@ -127,6 +127,13 @@ def make_qkv(B: int, H: int, Nq: int, Nk: int, d: int, dtype: str, seed: int,
     return q.to(t).contiguous(), k.to(t).contiguous(), v.to(t).contiguous()
 
 
+def make_grad_out(B: int, H: int, Nq: int, dv: int, dtype: str, seed: int):
+    """A seeded output gradient dO [B, H, Nq, dv], N(0,1) drawn on the CPU."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 7919)
+    return torch.randn((B, H, Nq, dv), generator=g, dtype=torch.float32).to(dtype_of(dtype)).contiguous()
+
+
 def make_workload_qkv(w: Workload):
     """Inputs of a named workload."""
     return make_qkv(w.B, w.H, w.Nq, w.Nk, w.d, w.dtype, w.seed, w.qk_scale)
