@@ -9,6 +9,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -50,7 +51,8 @@ struct DeviceInfo {
   bool probed = false;
   bool supported = false;
   int sms = 0;
-  bool smem_attr[2][2][3] = {};  // [d==128][bf16][unit, dual-unit, split kernel]
+  // [d==128][bf16][unit, dual-unit, split kernel]: the shared-memory attribute is set
+  std::atomic<bool> smem_attr[2][2][3] = {};
 };
 
 std::mutex g_dev_mutex;
@@ -199,8 +201,9 @@ bool encode_map(CUtensorMap* map, const void* ptr, int N, long long BH, int d, i
   return r == CUDA_SUCCESS;
 }
 
-// Per-thread cache of the last call's tensor maps: repeated calls on the same
-// buffers (the common case in a model loop) skip the ~µs host encode.
+// Per-thread cache of recent calls' tensor maps: repeated calls on the same
+// buffers (the common case in a model loop, and every chunk of the pipelined
+// host entry) skip the ~µs host encode.  Entries are replaced round robin.
 struct MapCache {
   const void* q = nullptr;
   const void* k = nullptr;
@@ -209,23 +212,48 @@ struct MapCache {
   long long BH = 0;
   CUtensorMap mq, mk, mv;
 };
-thread_local MapCache t_maps;
+constexpr int kMapCacheEntries = 16;
+struct MapCacheSet {
+  MapCache e[kMapCacheEntries];
+  int next = 0;
+};
+thread_local MapCacheSet t_maps;
+
+// The cached maps for these buffers and sizes, encoding them on a miss;
+// nullptr if an encode fails.
+const MapCache* cached_maps(const void* q, const void* k, const void* v, int Nq, int Nk,
+                            long long BH, int d, int dtype, int dev) {
+  MapCacheSet& set = t_maps;
+  for (const MapCache& mc : set.e)
+    if (mc.q == q && mc.k == k && mc.v == v && mc.Nq == Nq && mc.Nk == Nk && mc.d == d &&
+        mc.dtype == dtype && mc.dev == dev && mc.BH == BH)
+      return &mc;
+  MapCache& mc = set.e[set.next];
+  set.next = (set.next + 1) % kMapCacheEntries;
+  mc.q = nullptr;  // invalid until all three encodes succeed
+  if (!encode_map(&mc.mq, q, Nq, BH, d, dtype) || !encode_map(&mc.mk, k, Nk, BH, d, dtype) ||
+      !encode_map(&mc.mv, v, Nk, BH, d, dtype))
+    return nullptr;
+  mc.q = q; mc.k = k; mc.v = v;
+  mc.Nq = Nq; mc.Nk = Nk; mc.d = d; mc.dtype = dtype; mc.dev = dev; mc.BH = BH;
+  return &mc;
+}
 
 template <int D, bool BF16, bool SPLIT, bool DUAL>
 int launch_one(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo& info,
                cudaStream_t stream) {
   auto kernel = attn_sm100::attn_fwd_kernel<D, BF16, SPLIT, DUAL>;
   constexpr int smem = SmemLayout<D>::BYTES;
-  bool& attr = info.smem_attr[D == 128][BF16][SPLIT ? 2 : (DUAL ? 1 : 0)];
-  if (!attr) {
+  std::atomic<bool>& attr = info.smem_attr[D == 128][BF16][SPLIT ? 2 : (DUAL ? 1 : 0)];
+  if (!attr.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lock(g_dev_mutex);
-    if (!attr) {
+    if (!attr.load(std::memory_order_relaxed)) {
       if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
           cudaSuccess) {
         cudaGetLastError();
         return ATTN_ERR_CUDA;
       }
-      attr = true;
+      attr.store(true, std::memory_order_release);
     }
   }
   kernel<<<grid, NUM_THREADS, smem, stream>>>(maps.mq, maps.mk, maps.mv, prm);
@@ -257,16 +285,9 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   fill_plan(B, H, Nq, Nk, d, causal, info->sms, &plan);
   const long long BH = static_cast<long long>(B) * H;
 
-  MapCache& mc = t_maps;
-  if (mc.q != q || mc.k != k || mc.v != v || mc.Nq != Nq || mc.Nk != Nk || mc.d != d ||
-      mc.dtype != dtype || mc.dev != dev || mc.BH != BH) {
-    mc.q = nullptr;  // invalid until all three encodes succeed
-    if (!encode_map(&mc.mq, q, Nq, BH, d, dtype) || !encode_map(&mc.mk, k, Nk, BH, d, dtype) ||
-        !encode_map(&mc.mv, v, Nk, BH, d, dtype))
-      return ATTN_ERR_CUDA;
-    mc.q = q; mc.k = k; mc.v = v;
-    mc.Nq = Nq; mc.Nk = Nk; mc.d = d; mc.dtype = dtype; mc.dev = dev; mc.BH = BH;
-  }
+  const MapCache* maps = cached_maps(q, k, v, Nq, Nk, BH, d, dtype, dev);
+  if (maps == nullptr) return ATTN_ERR_CUDA;
+  const MapCache& mc = *maps;
 
   FwdParams prm;
   prm.o = o;
@@ -330,7 +351,7 @@ struct HostPipe {
   bool ready = false;
   std::mutex mu;
   cudaStream_t h2d = nullptr, comp = nullptr, d2h = nullptr;
-  cudaEvent_t start = nullptr, end = nullptr;
+  cudaEvent_t start = nullptr, end = nullptr, h2d_end = nullptr, comp_end = nullptr;
   cudaEvent_t in_done[kHostPipeMaxChunks] = {}, comp_done[kHostPipeMaxChunks] = {};
 };
 HostPipe g_host_pipe[kMaxDevices];
@@ -344,7 +365,9 @@ int host_pipe(int dev, HostPipe** out) {
               cudaStreamCreateWithFlags(&hp.comp, cudaStreamNonBlocking) == cudaSuccess &&
               cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) == cudaSuccess &&
               cudaEventCreateWithFlags(&hp.start, ef) == cudaSuccess &&
-              cudaEventCreateWithFlags(&hp.end, ef) == cudaSuccess;
+              cudaEventCreateWithFlags(&hp.end, ef) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.h2d_end, ef) == cudaSuccess &&
+              cudaEventCreateWithFlags(&hp.comp_end, ef) == cudaSuccess;
     for (int c = 0; ok && c < kHostPipeMaxChunks; ++c)
       ok = cudaEventCreateWithFlags(&hp.in_done[c], ef) == cudaSuccess &&
            cudaEventCreateWithFlags(&hp.comp_done[c], ef) == cudaSuccess;
@@ -458,11 +481,27 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
   if (st != ATTN_OK) return st;
   std::lock_guard<std::mutex> lock(hp->mu);
   const long long per = (bh + chunks - 1) / chunks;
+  // Joins the three library streams back into the caller's stream, so that
+  // work the caller enqueues afterwards (or a host wait before it frees or
+  // reuses the pinned buffers) follows everything this call enqueued -- on
+  // success and on every error path alike.
+  auto join = [&]() -> bool {
+    return cudaEventRecord(hp->h2d_end, hp->h2d) == cudaSuccess &&
+           cudaEventRecord(hp->comp_end, hp->comp) == cudaSuccess &&
+           cudaStreamWaitEvent(hp->d2h, hp->h2d_end, 0) == cudaSuccess &&
+           cudaStreamWaitEvent(hp->d2h, hp->comp_end, 0) == cudaSuccess &&
+           cudaEventRecord(hp->end, hp->d2h) == cudaSuccess &&
+           cudaStreamWaitEvent(s, hp->end, 0) == cudaSuccess;
+  };
   bool ok = cudaEventRecord(hp->start, s) == cudaSuccess &&
             cudaStreamWaitEvent(hp->h2d, hp->start, 0) == cudaSuccess &&
             cudaStreamWaitEvent(hp->comp, hp->start, 0) == cudaSuccess &&
             cudaStreamWaitEvent(hp->d2h, hp->start, 0) == cudaSuccess;
-  for (int c = 0; ok && c < chunks; ++c) {
+  if (!ok) {  // nothing of this call is enqueued yet
+    cudaGetLastError();
+    return ATTN_ERR_CUDA;
+  }
+  for (int c = 0; ok && st == ATTN_OK && c < chunks; ++c) {
     const long long h0 = c * per;
     const long long nh = (h0 + per <= bh) ? per : bh - h0;
     if (nh <= 0) break;
@@ -481,7 +520,7 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
                   static_cast<char*>(v_dev) + kvo, static_cast<char*>(o_dev) + qo,
                   lse_dev != nullptr ? lse_dev + lo : nullptr, static_cast<int>(nh), 1, Nq, Nk, d,
                   scale, causal, dtype, nullptr, 0, reinterpret_cast<attn_stream_t>(hp->comp));
-    if (st != ATTN_OK) return st;
+    if (st != ATTN_OK) break;
     ok = cudaEventRecord(hp->comp_done[c], hp->comp) == cudaSuccess &&
          cudaStreamWaitEvent(hp->d2h, hp->comp_done[c], 0) == cudaSuccess &&
          cudaMemcpyAsync(static_cast<char*>(o_host) + qo, static_cast<char*>(o_dev) + qo,
@@ -489,15 +528,15 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
          (!with_lse || cudaMemcpyAsync(lse_host + lo, lse_dev + lo, nh * Nq * sizeof(float),
                                        cudaMemcpyDeviceToHost, hp->d2h) == cudaSuccess);
   }
-  // the caller's stream continues after the last copy back (which itself
-  // followed every chunk's forward and copies in)
-  ok = ok && cudaEventRecord(hp->end, hp->d2h) == cudaSuccess &&
-       cudaStreamWaitEvent(s, hp->end, 0) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
-    return ATTN_ERR_CUDA;
+    st = ATTN_ERR_CUDA;
   }
-  return ATTN_OK;
+  if (!join()) {
+    cudaGetLastError();
+    if (st == ATTN_OK) st = ATTN_ERR_CUDA;
+  }
+  return st;
 }
 
 int attn_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, attn_plan_t* out) {
@@ -622,7 +661,3 @@ extern "C" int attn_fwd_noalloc(const void* q, const void* k, const void* v, voi
   return fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, ws,
                   kNoAllocScratchBytes, stream);
 }
-
-extern "C" {
-
-}  // extern "C"

@@ -53,11 +53,15 @@ constexpr int BLOCK_M = 128;     // query rows per Q tile (= TMEM lanes)
 constexpr int BLOCK_N = 128;     // keys per K / V tile
 // 12 warps = 3 warpgroups: two softmax warpgroups (warps 0-3, 4-7) and one
 // producer warpgroup (warp 8 issues the S MMAs, warp 9 the TMA loads of Q and
-// K, warp 10 the P V MMAs, warp 11 the TMA loads of V).  Launched at 168 registers per thread (the per-SM-sub-partition
-// limit for 3 warps each); the producer warpgroup then gives registers up
-// and the softmax warpgroups take them (2 * 128 * 200 + 128 * 96 = 63488, or
-// 2 * 128 * 208 + 128 * 88 = 64512, both <= 384 * 168), so the increase never
-// waits on registers that do not exist.
+// K, warp 10 the P V MMAs, warp 11 the TMA loads of V).  Launched at 168
+// registers per thread (the per-SM-sub-partition limit for 3 warps each); the
+// producer warpgroup then gives registers up and the softmax warpgroups take
+// them (2 * 128 * 200 + 128 * 96 = 63488, or 2 * 128 * 208 + 128 * 88 =
+// 64512, both <= 384 * 168), so the increase never waits on registers that
+// do not exist.  At 96 the MMA issuers of the unit-mode kernels keep one
+// descriptor word in local memory (an L1 hit per MMA issue, off the softmax's
+// critical path); giving them 104 removes that spill but measured 2-7 %
+// slower.
 constexpr int NUM_THREADS = 384;
 constexpr int MMA_WARP = 8;    // issues S = Q K^T
 constexpr int LOAD_WARP = 9;   // TMA loads of Q and K
@@ -170,8 +174,11 @@ struct SmemLayout {
   static constexpr int SYNC = DRAIN + 2;        // rendezvous of the 256 softmax threads
   static constexpr int NEVER = SYNC + 1;        // no thread ever arrives (test hook)
   static constexpr int NUM_BARS = NEVER + 1;
-  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // TMEM address, abort flag
-  static constexpr int BYTES = MISC_OFF + 16 + 1024;      // + slack to align the base to 1 KB
+  // TMEM address, abort flag, split flag, then (d = 64) the P V MMAs completed
+  // per tile, published by the P V issuer
+  static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;
+  static constexpr int PV_DONE_OFF = MISC_OFF + 16;
+  static constexpr int BYTES = PV_DONE_OFF + 8 + 1024;  // + slack to align the base to 1 KB
   // TMEM columns (512 allocated): S/P buffers, then O of tile 0 and tile 1
   static constexpr uint32_t TMEM_COLS = 512;
   static constexpr uint32_t S_COL = 0;           // + 128 * buffer
@@ -405,15 +412,27 @@ __device__ __forceinline__ bool last_use(const Unit& w, SeqPos s) {
 template <int D>
 __host__ __device__ constexpr bool kStaleMaxFirst() { return D == 64; }
 
-template <int D, bool BF16>
+// With the running max as it stands (STALE) x has no upper bound.  The
+// MUFU's 2^x overflows to +inf for x >= 128, which the caller's sum check
+// rejects, but the polynomial's exponent add wraps past x = 128 into small or
+// negative values that the sum would not reveal.  So a STALE call also
+// returns the largest x given to the polynomial, and the caller accepts the
+// row only if it stays below POLY_X_LIMIT, where the polynomial is exact to
+// its stated error (every x >= 15 then gives a P >= 2^15, which the sum
+// check rejects).  Without STALE, x <= RESCALE_LOG2 by construction.
+constexpr float POLY_X_LIMIT = 64.0f;
+
+template <int D, bool BF16, bool STALE>
 __device__ __forceinline__ float exp_row(const float (&s)[128], float sl2, float neg_m,
-                                         uint32_t (&pk)[64]) {
+                                         uint32_t (&pk)[64], float& xp_max) {
   float sum0 = 0.f, sum1 = 0.f;
+  float xm = -INFINITY;
 #pragma unroll
   for (int i = 0; i < 64; ++i) {
     float x0, x1, a, bb;
     fma2(x0, x1, s[2 * i], s[2 * i + 1], sl2, sl2, neg_m, neg_m);
     if (i % 16 < exp_poly_pairs<D>()) {
+      if constexpr (STALE) xm = max3(xm, x0, x1);
       exp2_poly2(a, bb, x0, x1);  // FMA pipe, in parallel with the MUFU ones
     } else {
       a = ex2_approx(x0);
@@ -422,7 +441,30 @@ __device__ __forceinline__ float exp_row(const float (&s)[128], float sl2, float
     add2(sum0, sum1, sum0, sum1, a, bb);
     pk[i] = pack2<BF16>(a, bb);
   }
+  xp_max = xm;
   return sum0 + sum1;
+}
+
+// Bounded wait until the 32-bit shared-memory counter at `addr` reaches
+// `target` (acquire load; same time limit and abort handling as wait_phase).
+__device__ __forceinline__ bool wait_count(uint32_t addr, uint32_t target, volatile int* abort_flag,
+                                           uint32_t site) {
+  uint32_t spins = 0;
+  uint64_t t0 = 0;
+  while (ld_acquire_shared(addr) < target) {
+    if ((++spins & 1023u) == 0) {
+      const uint64_t now = global_timer_ns();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > WAIT_LIMIT_NS) {
+        atomicCAS(&g_attn_status, 0u, 0x80000000u | site);
+        *abort_flag = 1;
+        return false;
+      }
+      if (*abort_flag) return false;
+    }
+  }
+  return true;
 }
 
 // Bounded wait on one mbarrier phase, fully inlined (a call here would make
@@ -492,6 +534,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(bar(L::SYNC), 2 * 128);
     mbar_init(bar(L::NEVER), 1);
     *abort_flag = 0;
+    reinterpret_cast<uint32_t*>(smem + L::PV_DONE_OFF)[0] = 0u;
+    reinterpret_cast<uint32_t*>(smem + L::PV_DONE_OFF)[1] = 0u;
     fence_mbarrier_init();
   }
   if (warp == LOAD_WARP && lane == 0) {
@@ -630,6 +674,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
       uint32_t pos = 0, g = 0, q_phase = 0;  // ring position of K_0 / V_0 of the item; score tile count
       uint32_t buf = 0, round = 0;           // g % NSB, g / NSB
+      uint32_t pv_ph0 = 0, pv_ph1 = 0, pv_n0 = 0, pv_n1 = 0;  // P V issuer: O_READY phases, counts
       bool ok = true;
       WorkCursor<SPLIT, DUAL> cur(p);
       Unit w;
@@ -767,6 +812,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 mma_commit(bar(L::PV_DONE + buf));
                 if (last_use<DUAL>(w, sp)) mma_commit(bar(L::V_EMPTY + st));
               }
+              // Wait for this P V and publish the tile's completed count: the
+              // softmax reads O (to rescale it or in the epilogue) only once the
+              // count covers every P it has handed over.  The next P V waits for
+              // the other tile's P anyway, so this wait costs the issue nothing.
+              {
+                const uint32_t ph = sp.t ? pv_ph1 : pv_ph0;
+                if (!warp_wait(bar(L::O_READY + sp.t), ph, SITE_MMA_P_FULL)) {
+                  ok = false;
+                  break;
+                }
+                if (sp.t) { pv_ph1 ^= 1u; ++pv_n1; } else { pv_ph0 ^= 1u; ++pv_n0; }
+                tc_fence_before();
+                if (leader)
+                  st_release_shared(smem_addr(smem + L::PV_DONE_OFF) + 4 * sp.t, sp.t ? pv_n1 : pv_n0);
+              }
             }
             ++g;
             if (++buf == static_cast<uint32_t>(NSB)) {
@@ -801,6 +861,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const uint32_t tO = tmem_base + lane_off + L::O_COL + D * t;
     const float sl2 = p.scale_log2;
     uint32_t o_phase = 0, sk = 0;
+    uint32_t pv_handed = 0;  // P tiles of this Q tile handed to the P V MMA so far
     uint32_t s_parity = 0;  // bit b: parity of the next S_FULL(b, t) phase this warpgroup waits for
     bool ok = true;
     volatile int* last_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 8);
@@ -866,17 +927,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             // P = 2^(s * scale * log2 e - m), packed two keys per 32-bit word
             // (even key in the low half).  After the first tile the running
             // max m is tried as it stands: the sum of the tile's P bounds every
-            // P, so if it stays below 2^15 no P overflows a 16-bit float and
-            // the result is exact with the stale max, and the row max is
-            // never computed.  Otherwise (or on the first tile) S is read
-            // again and the row max decides, as below.  P is written to TMEM
-            // only after that decision, so S is still there to be read again.
+            // P, so if it stays below 2^15 (and every exponent given to the
+            // polynomial lies in its valid range, see exp_row) no P overflows
+            // a 16-bit float and the result is exact with the stale max, and
+            // the row max is never computed.  Otherwise (or on the first
+            // tile) S is read again and the row max decides, as below.  P is
+            // written to TMEM only after that decision, so S is still there
+            // to be read again.
             uint32_t pk[64];
             float tsum = 0.f;
             bool settled = false;
             if (j > 0) {
-              tsum = exp_row<D, BF16>(s, sl2, -m, pk);
-              settled = __all_sync(0xffffffffu, tsum < 32768.f);
+              float xp_max;
+              tsum = exp_row<D, BF16, true>(s, sl2, -m, pk, xp_max);
+              settled = __all_sync(0xffffffffu, tsum < 32768.f && xp_max < POLY_X_LIMIT);
               if (!settled) load_s();
             }
             if (!settled) {
@@ -902,7 +966,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               m_new = raise ? m_cand : m;
               const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
               alpha = raise ? ex2_approx(m - m_use) : 1.f;
-              tsum = exp_row<D, BF16>(s, sl2, -m_use, pk);
+              float xp_unused;
+              tsum = exp_row<D, BF16, false>(s, sl2, -m_use, pk, xp_unused);
             }
             tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
             tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
@@ -978,15 +1043,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // O_t may only be touched once the previous P V of this tile is
           // done: with split issue that is its own signal; with in-order issue
           // (two S buffers) the S just read was queued behind that P V.
-          if (j > 0) {
+          if (j > 0 && __any_sync(0xffffffffu, raise)) {
             if constexpr (NSB > 2) {
-              ok = wait_phase(bar(L::O_READY + t), o_phase, abort_flag, SITE_SOFTMAX_O_READY);
+              ok = wait_count(smem_addr(smem + L::PV_DONE_OFF) + 4 * t, pv_handed, abort_flag,
+                              SITE_SOFTMAX_O_READY);
               ok = __all_sync(0xffffffffu, ok);
               if (!ok) break;
-              o_phase ^= 1;
               tc_fence_after();
             }
-            if (__any_sync(0xffffffffu, raise)) {
+            {
 #pragma unroll
               for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t o[32];
@@ -1006,6 +1071,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tmem_wait_st();
           tc_fence_before();
           mbar_arrive(bar(L::P_FULL + b));
+          ++pv_handed;
         }
         if (!ok) break;
 
@@ -1013,10 +1079,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const bool in_range = row < p.Nq;
         float lse_self = 0.f, inv_self = 0.f;  // this piece's statistics, for the merge
         if (n > 0) {
-          ok = wait_phase(bar(L::O_READY + t), o_phase, abort_flag, SITE_SOFTMAX_O_READY);
+          if constexpr (NSB > 2) {
+            ok = wait_count(smem_addr(smem + L::PV_DONE_OFF) + 4 * t, pv_handed, abort_flag,
+                            SITE_SOFTMAX_O_READY);
+          } else {
+            ok = wait_phase(bar(L::O_READY + t), o_phase, abort_flag, SITE_SOFTMAX_O_READY);
+            o_phase ^= 1;
+          }
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
-          o_phase ^= 1;
           tc_fence_after();
           const float inv_l = 1.f / l;
           const float lse_row = (m + lg2_approx(l)) * 0.69314718055994531f;

@@ -82,6 +82,16 @@ __device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Release store / acquire load of a 32-bit shared-memory word (CTA scope).
+__device__ __forceinline__ void st_release_shared(uint32_t addr, uint32_t v) {
+  asm volatile("st.release.cta.shared::cta.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
+__device__ __forceinline__ uint32_t ld_acquire_shared(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.acquire.cta.shared::cta.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -294,7 +304,9 @@ __device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, f
 // (minimax in relative error, max 7.5e-5, coefficients from
 // fit_exp2_poly.py); 2^j is applied by adding j to the exponent field.  x is
 // clamped at -126 so the exponent add never underflows; results below
-// 2^-126 are returned as tiny normal or subnormal values, not zero.
+// 2^-126 are returned as tiny normal or subnormal values, not zero.  There is
+// no clamp above: for x >= 128 the exponent add wraps into the sign bit, so
+// callers must keep x below 128 or check the largest x they pass.
 __device__ __forceinline__ void exp2_poly2(float& y0, float& y1, float x0, float x1) {
   constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
   constexpr float c0 = 0.9999280571937561f, c1 = 0.6932609677314758f;

@@ -18,12 +18,16 @@
  *   - causal != 0 applies the top-left aligned mask: query i sees key j iff j <= i (the
  *     convention of torch's is_causal).  Every query row sees at least key 0.
  *   - scale is the factor applied to Q K^T; the usual value is 1/sqrt(d).
- *   - All memory is owned by the caller.  The library allocates nothing per call.
+ *   - All memory is owned by the caller.  The library allocates nothing per call.  The one
+ *     exception is attn_fwd_noalloc, which uses a fixed scratch array inside the library
+ *     (see its declaration).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; 0 = legacy default stream).  A
  *     return of ATTN_OK means the arguments were valid and the kernel was enqueued.
  *   - No fallback path exists: an unsupported input returns an error code; nothing is
  *     computed a different way.
- *   - Thread safety: calls from several host threads are safe.
+ *   - Thread safety: calls from several host threads are safe, except that calls of
+ *     attn_fwd_noalloc that overlap on the GPU race on its shared scratch array (see its
+ *     declaration).
  */
 #ifndef ATTN_SM100_ATTN_H_
 #define ATTN_SM100_ATTN_H_
@@ -211,7 +215,11 @@ int attn_fwd_stall_test(const void* q, const void* k, const void* v, void* o, fl
  *
  * Argument rules and error codes are those of attn_fwd; every host and device pointer
  * except the lse pair must be non-NULL.  workspace / workspace_bytes are optional (NULL, 0)
- * and act as in attn_fwd_ws.  Nothing is allocated per call.
+ * and act as in attn_fwd_ws.  Nothing is allocated per call.  Argument errors are found
+ * before anything is enqueued.  If a CUDA call fails after some copies were enqueued, the
+ * call still orders `stream` after everything it enqueued before returning the error, so a
+ * synchronisation of `stream` is enough before the host buffers are freed or reused; the
+ * outputs are then invalid.
  */
 int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, void* o_host,
                   float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
