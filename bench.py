@@ -151,6 +151,25 @@ class ClockSampler(threading.Thread):
         return out
 
 
+L2_NOTE = "flushed before every timed call (256 MiB write)"
+GRAPH_CALLS = {"yolo_c2psa_20x20": 2000, "yolo_neck_40x40_b16": 200,
+               "yolo_highres_80x80_b16": 20, "llm_causal_2048": 20, "long_context_32k": 5}
+
+
+def bench_config(w, world: int) -> dict:
+    """The config dict of the JSON line; both arms print exactly this for the same workload."""
+    return dict(w.as_config(), l2=L2_NOTE,
+                parallelism=f"dp{world} over (batch, head) slices, no collective")
+
+
+def percentiles(values):
+    """Median, p10, p90 and mean of a list of per-call times."""
+    import numpy as np
+    a = np.asarray(values, dtype=np.float64)
+    return {"median": float(np.median(a)), "p10": float(np.percentile(a, 10)),
+            "p90": float(np.percentile(a, 90)), "mean": float(a.mean())}
+
+
 def rank_seed(w, rank: int) -> int:
     """Seed of rank ``rank``'s own copy of the workload (weak scaling: one slice per rank)."""
     return w.seed + 1000 * rank
@@ -232,7 +251,8 @@ def run_reference(args, w):
         "warmup": args.warmup, "ms_per_step": tot_t / args.steps * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1))",
-        "config": dict(w.as_config(), parallelism="host cores, rank 0 only"),
+        "config": bench_config(w, int(os.environ.get("WORLD_SIZE", args.gpus))),
+        "reference_run": "float64 oracle on the host cores of rank 0; other ranks do no work",
         "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0,
@@ -376,7 +396,8 @@ def main():
     per_workload = None
     cpu = None
     if rank == 0 and world == 1 and not args.no_per_workload:
-        per_workload = context_timings(attn, torch, dev, peaks)
+        per_workload = context_timings(attn, torch, dev, peaks, steps=args.steps,
+                                       warmup=args.warmup, device_index=local)
     if rank == 0:
         flops, dt, done = time_oracle_sample(w, q, k, v, budget_s=args.cpu_budget)
         cpu = {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": blas_threads() or cpu_cores(),
@@ -391,8 +412,8 @@ def main():
             "us_per_call": round(ms_per_step * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic (seeded N(0,1), recipe in seeded_inputs)",
-            "config": dict(w.as_config(), l2="flushed before every timed step (256 MiB write)",
-                           parallelism=f"dp{world} over (batch, head) slices, no collective"),
+            "config": bench_config(w, world),
+            "us_per_call_stats": {k: round(v * 1e3, 2) for k, v in percentiles(kernel_ms).items()},
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": round(e2e_value, 3), "unit": "TFLOPS",
@@ -413,8 +434,41 @@ def main():
     return 0
 
 
-def context_timings(attn, torch, dev, peaks, steps=10):
-    """µs/call, TFLOPS and roofline fraction of every workload (L2 flushed each call)."""
+def graph_per_call_us(attn, torch, w, q, k, v, o, lse, ws, calls: int, replays: int = 10):
+    """Per-call µs of ``calls`` back-to-back forwards captured in one CUDA graph (L2 warm).
+
+    Launch overhead is amortised over the graph; each call is still its own
+    kernel launch (nothing is merged).  Returns the median over ``replays``.
+    """
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):  # warm-up on the capture stream, outside the graph
+        for _ in range(3):
+            attn.forward(q, k, v, causal=w.causal, out=o, lse=lse, workspace=ws)
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for _ in range(calls):
+            attn.forward(q, k, v, causal=w.causal, out=o, lse=lse, workspace=ws)
+    g.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(replays):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) * 1e3 / calls)
+    del g
+    return statistics.median(times)
+
+
+def context_timings(attn, torch, dev, peaks, steps=50, warmup=5, device_index=0):
+    """Every workload: cold single-call µs (L2 flushed each call; median, p10, p90), TFLOPS and
+    roofline fraction of the median, the clocks seen meanwhile, and a CUDA-graph-replayed warm
+    per-call figure."""
     from seeded_inputs import WORKLOADS, make_workload_qkv
     out = {}
     flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
@@ -423,24 +477,38 @@ def context_timings(attn, torch, dev, peaks, steps=10):
         o = torch.empty_like(q)
         lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
         ws = attn.workspace_for(q, k, w.causal)
-        for _ in range(3):
-            attn.forward(q, k, v, causal=w.causal, out=o, lse=lse, workspace=ws)
-        times = []
-        for _ in range(steps):
+        for _ in range(max(3, warmup)):
             flush.zero_()
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            attn.forward(q, k, v, causal=w.causal, out=o, lse=lse, workspace=ws)
+        torch.cuda.synchronize()
+        sampler = ClockSampler(device_index)
+        sampler.start()
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(steps)]
+        for e0, e1 in evs:
+            flush.zero_()
             e0.record()
             attn.forward(q, k, v, causal=w.causal, out=o, lse=lse, workspace=ws)
             e1.record()
-            torch.cuda.synchronize()
-            times.append(e0.elapsed_time(e1))
-        us = statistics.median(times) * 1e3
+        torch.cuda.synchronize()
+        times = [e0.elapsed_time(e1) * 1e3 for e0, e1 in evs]
+        calls = GRAPH_CALLS.get(w.name, 20)
+        graph_us = graph_per_call_us(attn, torch, w, q, k, v, o, lse, ws, calls)
+        sampler.stop()
+        st = percentiles(times)
+        us = st["median"]
         r = roofline(w, us * 1e-6, peaks)
-        out[w.name] = {"us_per_call": round(us, 2), "split": ws is not None,
+        out[w.name] = {"us_per_call": round(us, 2),
+                       "us_p10": round(st["p10"], 2), "us_p90": round(st["p90"], 2),
+                       "calls": steps, "split": ws is not None,
                        "tflops": round(w.flops / (us * 1e-6) / 1e12, 2),
                        "bound": r["bound"], "frac": r["frac"],
-                       "frac_of_sustained": roofline(w, us * 1e-6, peaks, sustained=True)["frac"]}
+                       "frac_of_sustained": roofline(w, us * 1e-6, peaks, sustained=True)["frac"],
+                       "graph_warm_us_per_call": round(graph_us, 2), "graph_calls": calls,
+                       "graph_warm_frac": roofline(w, graph_us * 1e-6, peaks)["frac"],
+                       "clocks": sampler.summary()}
         del q, k, v, o, lse
+        torch.cuda.empty_cache()
     return out
 
 

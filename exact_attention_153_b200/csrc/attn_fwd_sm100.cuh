@@ -148,8 +148,12 @@ struct SmemLayout {
   // separate K and V rings, filled in the order the MMA warp consumes them
   static constexpr int K_STAGES = (D == 64) ? 4 : 3;
   static constexpr int V_STAGES = (D == 64) ? 4 : 2;
+  // Q: slots of two tiles.  Two slots at d = 64, so the next item's Q tiles
+  // load while the current item runs and its first S does not wait for them;
+  // one at d = 128, where shared memory has no room for a second.
+  static constexpr int Q_SLOTS = (D == 64) ? 2 : 1;
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + 2 * TILE_BYTES;
+  static constexpr int K_OFF = Q_OFF + Q_SLOTS * 2 * TILE_BYTES;
   static constexpr int V_OFF = K_OFF + K_STAGES * TILE_BYTES;
   static constexpr int BAR_OFF = V_OFF + V_STAGES * TILE_BYTES;
   // S/P buffers in TMEM: three at d = 64 (so a tile's next S is computed
@@ -161,12 +165,12 @@ struct SmemLayout {
   static constexpr int K_EMPTY = K_FULL + K_STAGES;
   static constexpr int V_FULL = K_EMPTY + K_STAGES;
   static constexpr int V_EMPTY = V_FULL + V_STAGES;
-  static constexpr int Q_FULL = V_EMPTY + V_STAGES;
-  static constexpr int Q_EMPTY = Q_FULL + 1;
+  static constexpr int Q_FULL = V_EMPTY + V_STAGES;  // + slot
+  static constexpr int Q_EMPTY = Q_FULL + Q_SLOTS;   // + slot
   // S ready: one barrier per (buffer, tile), so each softmax warpgroup only
   // waits on phases it alone consumes (a per-buffer barrier shared by both
   // tiles could be two phases behind a warpgroup that skipped an item).
-  static constexpr int S_FULL = Q_EMPTY + 1;       // + 2 * buffer + tile
+  static constexpr int S_FULL = Q_EMPTY + Q_SLOTS;  // + 2 * buffer + tile
   static constexpr int P_FULL = S_FULL + 2 * NSB;  // + buffer (one waiter: the MMA warp)
   static constexpr int O_READY = P_FULL + NSB; // + tile: one phase per P V MMA of the tile
   static constexpr int PV_DONE = O_READY + 2;  // + buffer: P V of that buffer finished
@@ -473,6 +477,9 @@ __device__ __forceinline__ bool wait_count(uint32_t addr, uint32_t target, volat
 // honour_abort, once another role has aborted.
 __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                            uint32_t site, bool honour_abort = true) {
+  // a phase that has already completed is found by the non-blocking test;
+  // only an open phase enters the (suspending) try_wait loop
+  if (mbar_test_wait(bar, parity)) return true;
   uint32_t spins = 0;
   uint64_t t0 = 0;
   while (!mbar_try_wait(bar, parity)) {
@@ -519,8 +526,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar(L::V_FULL + s), 1);
       mbar_init(bar(L::V_EMPTY + s), 1);
     }
-    mbar_init(bar(L::Q_FULL), 1);
-    mbar_init(bar(L::Q_EMPTY), 1);
+    for (int s = 0; s < L::Q_SLOTS; ++s) {
+      mbar_init(bar(L::Q_FULL + s), 1);
+      mbar_init(bar(L::Q_EMPTY + s), 1);
+    }
     for (int b = 0; b < NSB; ++b) {
       mbar_init(bar(L::S_FULL + 2 * b), 1);
       mbar_init(bar(L::S_FULL + 2 * b + 1), 1);
@@ -591,19 +600,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               ok = false;
               break;
             }
-            if (items_done > 0) {
-              ok = warp_wait(bar(L::Q_EMPTY), (items_done - 1) & 1, SITE_LOAD_Q_EMPTY);
+            // item i uses Q slot i % Q_SLOTS, free again once the S MMAs of
+            // item i - Q_SLOTS have completed
+            const uint32_t qs = items_done % L::Q_SLOTS;
+            if (items_done >= static_cast<uint32_t>(L::Q_SLOTS)) {
+              ok = warp_wait(bar(L::Q_EMPTY + qs), (items_done / L::Q_SLOTS - 1) & 1,
+                             SITE_LOAD_Q_EMPTY);
               if (!ok) break;
             }
             if (leader) {
-              mbar_arrive_expect_tx(bar(L::Q_FULL), 2 * L::TILE_BYTES);
+              mbar_arrive_expect_tx(bar(L::Q_FULL + qs), 2 * L::TILE_BYTES);
 #pragma unroll
               for (int t = 0; t < 2; ++t)
 #pragma unroll
                 for (int h = 0; h < L::HALVES; ++h)
-                  tma_load_3d(q_smem + t * L::TILE_BYTES + h * L::HALF_BYTES, &tm_q,
-                              bar(L::Q_FULL), h * 64, (DUAL && t) ? w.q1 : w.q0 + t * BLOCK_M,
-                              (DUAL && t) ? w.bh1 : w.bh);
+                  tma_load_3d(q_smem + (2 * qs + t) * L::TILE_BYTES + h * L::HALF_BYTES, &tm_q,
+                              bar(L::Q_FULL + qs), h * 64,
+                              (DUAL && t) ? w.q1 : w.q0 + t * BLOCK_M, (DUAL && t) ? w.bh1 : w.bh);
             }
             __syncwarp();
           }
@@ -633,8 +646,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // Every issued load must have landed before the CTA may exit.
       for (uint32_t i = pos > static_cast<uint32_t>(stages) ? pos - stages : 0; i < pos; ++i)
         wait_phase(bar(full0 + i % stages), (i / stages) & 1, abort_flag, SITE_DRAIN, false);
-      if (is_k && items_done > 0)
-        wait_phase(bar(L::Q_FULL), (items_done - 1) & 1, abort_flag, SITE_DRAIN, false);
+      if (is_k) {
+        for (uint32_t i = items_done > static_cast<uint32_t>(L::Q_SLOTS) ? items_done - L::Q_SLOTS : 0;
+             i < items_done; ++i)
+          wait_phase(bar(L::Q_FULL + i % L::Q_SLOTS), (i / L::Q_SLOTS) & 1, abort_flag, SITE_DRAIN,
+                     false);
+      }
       __syncwarp();
     } else if (warp == MMA_WARP || warp == PV_WARP) {
       // ----------------------------------------------------------- MMA issuers
@@ -672,7 +689,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       } else {
       const bool is_s = (warp == MMA_WARP);
 
-      uint32_t pos = 0, g = 0, q_phase = 0;  // ring position of K_0 / V_0 of the item; score tile count
+      uint32_t pos = 0, g = 0;  // ring position of K_0 / V_0 of the item; score tile count
+      uint32_t items = 0;       // items begun (the Q slot is items % Q_SLOTS)
       uint32_t buf = 0, round = 0;           // g % NSB, g / NSB
       uint32_t pv_ph0 = 0, pv_ph1 = 0, pv_n0 = 0, pv_n1 = 0;  // P V issuer: O_READY phases, counts
       bool ok = true;
@@ -687,10 +705,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               ok = false;
               break;
             }
-            ok = warp_wait(bar(L::Q_FULL), q_phase, SITE_MMA_Q_FULL);
+            ok = warp_wait(bar(L::Q_FULL + items % L::Q_SLOTS), (items / L::Q_SLOTS) & 1,
+                           SITE_MMA_Q_FULL);
             if (!ok) break;
-            q_phase ^= 1;
           }
+          const uint32_t q_slot = items % L::Q_SLOTS;
+          const uint64_t q_item = q_desc + q_slot * static_cast<uint32_t>((2 * L::TILE_BYTES) >> 4);
           int ready_j = -1;
           if constexpr (!kSplit) {
             // in-order issue: S(0), S(1), then P V(k) followed by S(k + 2)
@@ -707,7 +727,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 k_ready = slot;
               }
               const uint32_t b = (g + k) % NSB;
-              const uint64_t a = q_desc + static_cast<uint32_t>(sp.t * (L::TILE_BYTES >> 4));
+              const uint64_t a = q_item + static_cast<uint32_t>(sp.t * (L::TILE_BYTES >> 4));
               const uint64_t bd = k_desc + st * static_cast<uint32_t>(L::TILE_BYTES >> 4);
               if (leader) {
 #pragma unroll
@@ -776,7 +796,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 break;
               }
               tc_fence_after();
-              const uint64_t a = q_desc + static_cast<uint32_t>(sp.t * (L::TILE_BYTES >> 4));
+              const uint64_t a = q_item + static_cast<uint32_t>(sp.t * (L::TILE_BYTES >> 4));
               const uint64_t bd = k_desc + st * static_cast<uint32_t>(L::TILE_BYTES >> 4);
               if (leader) {
 #pragma unroll
@@ -837,7 +857,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (!ok) break;
           // every S of the item has been issued: the Q tiles may be replaced
           // once those MMAs complete
-          if (is_s && leader) mma_commit(bar(L::Q_EMPTY));
+          if (is_s && leader) mma_commit(bar(L::Q_EMPTY + q_slot));
+          ++items;
           __syncwarp();
           pos += DUAL ? w.nmax * w.kvs : w.nmax;
         }

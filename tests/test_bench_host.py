@@ -37,3 +37,23 @@ def test_recorded_traffic_only_for_current_sources(tmp_path, monkeypatch):
     doc["kernel_source_sha"] = "0" * 16  # counters taken on other sources
     path.write_text(json.dumps(doc))
     assert bench.recorded_traffic("yolo_neck_40x40_b16") is None
+
+
+def test_both_arms_print_the_same_config(capsys, monkeypatch):
+    """The reference arm's config dict is the GPU arm's, key for key."""
+    import argparse
+    w = workload("yolo_c2psa_20x20")
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    args = argparse.Namespace(gpus=1, steps=1, warmup=0)
+    monkeypatch.setattr(bench, "time_oracle_sample",
+                        lambda *a, **k: (w.flops / (w.B * w.H), 0.5, 1))
+    bench.run_reference(args, w)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.bench_config(w, 1)
+
+
+def test_percentiles():
+    st = bench.percentiles([float(x) for x in range(1, 101)])
+    assert st["median"] == 50.5 and abs(st["p10"] - 10.9) < 1e-9 and abs(st["p90"] - 90.1) < 1e-9
