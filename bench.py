@@ -394,10 +394,12 @@ def main():
     roof["algorithmic_bytes_per_launch"] = w.bytes
 
     per_workload = None
+    backward = None
     cpu = None
     if rank == 0 and world == 1 and not args.no_per_workload:
         per_workload = context_timings(attn, torch, dev, peaks, steps=args.steps,
                                        warmup=args.warmup, device_index=local)
+        backward = backward_timings(attn, torch, dev, peaks, warmup=args.warmup)
     if rank == 0:
         flops, dt, done = time_oracle_sample(w, q, k, v, budget_s=args.cpu_budget)
         cpu = {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": blas_threads() or cpu_cores(),
@@ -428,10 +430,55 @@ def main():
         }
         if per_workload is not None:
             line["per_workload"] = per_workload
+        if backward is not None:
+            line["backward"] = backward
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
     return 0
+
+
+def backward_flops(w) -> float:
+    """Algorithmic FLOPs of the backward: five N x N x d contractions (S, dP, dV, dK, dQ)."""
+    f = 10.0 * w.B * w.H * w.Nq * w.Nk * w.d
+    return f / 2.0 if w.causal else f
+
+
+def backward_timings(attn, torch, dev, peaks, steps=20, warmup=3):
+    """µs/call (L2 flushed before each call; median, p10, p90) and TFLOP/s of attn_bwd
+    (row pass, main pass, dQ conversion) on every workload."""
+    from seeded_inputs import WORKLOADS, make_grad_out, make_workload_qkv
+    out = {}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for w in WORKLOADS:
+        q, k, v = (t.to(dev) for t in make_workload_qkv(w))
+        do = make_grad_out(w.B, w.H, w.Nq, w.d, w.dtype, w.seed).to(dev)
+        o, lse = attn.forward(q, k, v, causal=w.causal)
+        ws = torch.empty(attn.attn_bwd_workspace_size(w.B, w.H, w.Nq, w.Nk, w.d),
+                         dtype=torch.uint8, device=dev)
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+        for _ in range(max(3, warmup)):
+            attn.backward(q, k, v, o, lse, do, causal=w.causal, workspace=ws, out=grads)
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            attn.backward(q, k, v, o, lse, do, causal=w.causal, workspace=ws, out=grads)
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) * 1e3)
+        st = percentiles(times)
+        us = st["median"]
+        tf = backward_flops(w) / (us * 1e-6) / 1e12
+        out[w.name] = {"us_per_call": round(us, 2), "us_p10": round(st["p10"], 2),
+                       "us_p90": round(st["p90"], 2), "tflops": round(tf, 2),
+                       "frac": round(tf / peaks["bf16_tflops"], 4), "bound": "tensor",
+                       "launches": 3}
+        del q, k, v, do, o, lse, ws, grads
+        torch.cuda.empty_cache()
+    return out
 
 
 def graph_per_call_us(attn, torch, w, q, k, v, o, lse, ws, calls: int, replays: int = 10):

@@ -22,7 +22,7 @@ __all__ = [
     "ATTN_FP16", "ATTN_BF16", "AttnError", "lib", "library_path", "attn_fwd", "attn_fwd_host",
     "attn_plan", "attn_get_device_status", "attn_strerror", "attn_version", "forward",
     "forward_host", "STATUS_NAMES", "attn_fwd_ws", "attn_workspace_size", "workspace_for",
-    "attn_fwd_noalloc",
+    "attn_fwd_noalloc", "attn_bwd", "attn_bwd_workspace_size", "backward",
 ]
 
 ATTN_FP16 = 0
@@ -31,6 +31,7 @@ STATUS_NAMES = {
     0: "ATTN_OK", 1: "ATTN_ERR_NULL", 2: "ATTN_ERR_SHAPE", 3: "ATTN_ERR_HEAD_DIM",
     4: "ATTN_ERR_DTYPE", 5: "ATTN_ERR_ALIGN", 6: "ATTN_ERR_SCALE", 7: "ATTN_ERR_ARCH",
     8: "ATTN_ERR_CUDA", 9: "ATTN_ERR_DEVICE_TIMEOUT", 10: "ATTN_ERR_SCRATCH_LIMIT",
+    11: "ATTN_ERR_WORKSPACE",
 }
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +87,10 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_stall_test.restype = i
         L.attn_fwd_host.argtypes = [vp] * 11 + [ctypes.c_size_t, i, i, i, i, i, f, i, i, vp]
         L.attn_fwd_host.restype = i
+        L.attn_bwd.argtypes = [vp] * 9 + [i, i, i, i, i, f, i, i, vp, ctypes.c_size_t, vp]
+        L.attn_bwd.restype = i
+        L.attn_bwd_workspace_size.argtypes = [i, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
+        L.attn_bwd_workspace_size.restype = i
         L.attn_plan.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(_Plan)]
         L.attn_plan.restype = i
         L.attn_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
@@ -126,6 +131,22 @@ def attn_fwd_stall_test(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, 
     """Raw ``attn_fwd_stall_test``: the failure-path test hook (see include/attn.h)."""
     return lib().attn_fwd_stall_test(q, k, v, o, lse, B, H, Nq, Nk, d, float(scale),
                                      int(causal), dtype, workspace, ws_bytes, stall_site, stream)
+
+
+def attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, Nq, Nk, d, scale, causal, dtype, workspace,
+             ws_bytes, stream) -> int:
+    """Raw ``attn_bwd``: pointers and the stream handle as Python ints."""
+    return lib().attn_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, H, Nq, Nk, d, float(scale),
+                          int(causal), dtype, workspace, ws_bytes, stream)
+
+
+def attn_bwd_workspace_size(B, H, Nq, Nk, d) -> int:
+    """Workspace bytes ``attn_bwd`` needs for these sizes."""
+    n = ctypes.c_size_t(0)
+    st = lib().attn_bwd_workspace_size(B, H, Nq, Nk, d, ctypes.byref(n))
+    if st != 0:
+        raise AttnError(st, "attn_bwd_workspace_size")
+    return n.value
 
 
 def attn_workspace_size(B, H, Nq, Nk, d, causal) -> int:
@@ -258,3 +279,32 @@ def forward_host(q_h, k_h, v_h, o_h, lse_h, q_d, k_d, v_d, o_d, lse_d, causal=Fa
                        B, H, Nq, Nk, d, scale, causal, _dtype_code(q_h), _stream_handle(stream))
     if st != 0:
         raise AttnError(st, "attn_fwd_host")
+
+
+def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
+             stream=None, workspace=None, out=None):
+    """Gradients (dq, dk, dv) of the forward for the output gradient ``dout``.
+
+    ``o`` and ``lse`` are the forward's outputs for these inputs.  A workspace
+    of ``attn_bwd_workspace_size`` bytes is allocated when none is given.
+    """
+    import torch
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    for name, t in (("q", q), ("k", k), ("v", v), ("o", o), ("dout", dout), ("lse", lse)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    if workspace is None:
+        workspace = torch.empty(attn_bwd_workspace_size(B, H, Nq, Nk, d), dtype=torch.uint8,
+                                device=q.device)
+    dq, dk, dv = out if out is not None else (torch.empty_like(q), torch.empty_like(k),
+                                              torch.empty_like(v))
+    st = attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                  dout.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), B, H, Nq, Nk, d,
+                  scale, causal, _dtype_code(q), workspace.data_ptr(),
+                  workspace.numel() * workspace.element_size(), _stream_handle(stream))
+    if st != 0:
+        raise AttnError(st, "attn_bwd")
+    return dq, dk, dv

@@ -16,6 +16,7 @@
 #include <mutex>
 
 #include "attn.h"
+#include "attn_bwd_sm100.cuh"
 #include "attn_fwd_sm100.cuh"
 
 namespace {
@@ -585,6 +586,7 @@ const char* attn_strerror(int status) {
     case ATTN_ERR_CUDA: return "a CUDA call failed (no usable device, encode or launch error)";
     case ATTN_ERR_DEVICE_TIMEOUT: return "a kernel gave up on a bounded internal wait; its output is invalid";
     case ATTN_ERR_SCRATCH_LIMIT: return "the problem needs more scratch than attn_fwd_noalloc's fixed 24 MiB";
+    case ATTN_ERR_WORKSPACE: return "the workspace is NULL, smaller than attn_bwd_workspace_size or not 16-byte aligned";
     default: return "unknown status";
   }
 }
@@ -592,6 +594,131 @@ const char* attn_strerror(int status) {
 int attn_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward: row pass, main pass, dQ conversion.
+// ---------------------------------------------------------------------------
+namespace {
+
+// fp32 dQ accumulator [BH][Nq][d], then lse in base 2 and D, each [BH][Nq_pad].
+size_t bwd_workspace_bytes(long long BH, int Nq, int d) {
+  const size_t nq_pad = static_cast<size_t>(ceil_div(Nq, BLOCK_M)) * BLOCK_M;
+  return static_cast<size_t>(BH) * Nq * d * 4 + 2 * static_cast<size_t>(BH) * nq_pad * 4;
+}
+
+struct BwdMapCache {
+  const void* dout = nullptr;
+  int Nq = 0, d = 0, dtype = -1, dev = -1;
+  long long BH = 0;
+  CUtensorMap m;
+};
+thread_local BwdMapCache t_do_map;
+
+std::atomic<bool> g_bwd_attr[kMaxDevices][2][2];  // [dev][d == 128][bf16]
+
+template <int D, bool BF16>
+int bwd_launch(const MapCache& maps, const CUtensorMap& m_do, const void* o, const void* dout,
+               const float* lse, void* dq, const attn_sm100::BwdParams& prm, int dev, int sms,
+               cudaStream_t stream) {
+  using L = attn_sm100::BwdSmem<D>;
+  auto main_kernel = attn_sm100::bwd_main_kernel<D, BF16>;
+  std::atomic<bool>& attr = g_bwd_attr[dev][D == 128][BF16];
+  if (!attr.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!attr.load(std::memory_order_relaxed)) {
+      if (cudaFuncSetAttribute(main_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               L::BYTES) != cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+      }
+      attr.store(true, std::memory_order_release);
+    }
+  }
+  const long long BH = prm.BH;
+  const long long prep_rows = BH * prm.nq_pad;
+  const long long prep_blocks_needed = (prep_rows + 31) / 32;  // 32 rows per 256-thread block
+  const int prep_blocks = static_cast<int>(prep_blocks_needed < 16LL * sms ? prep_blocks_needed : 16LL * sms);
+  attn_sm100::bwd_prep_kernel<D, BF16><<<prep_blocks, 256, 0, stream>>>(
+      static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), lse,
+      const_cast<float*>(prm.lse2), const_cast<float*>(prm.dsum), prm.dq_acc, prm.Nq, prm.nq_pad, BH);
+  const long long grid = static_cast<long long>(prm.nk_tiles) * BH;
+  main_kernel<<<static_cast<unsigned int>(grid), attn_sm100::BWD_THREADS, L::BYTES, stream>>>(
+      maps.mq, maps.mk, maps.mv, m_do, prm);
+  const long long n4 = BH * prm.Nq * (D / 4);
+  const long long dq_blocks_needed = (n4 + 255) / 256;
+  const int dq_blocks = static_cast<int>(dq_blocks_needed < 16LL * sms ? dq_blocks_needed : 16LL * sms);
+  attn_sm100::bwd_dq_kernel<BF16><<<dq_blocks, 256, 0, stream>>>(prm.dq_acc,
+                                                                 static_cast<uint16_t*>(dq), n4,
+                                                                 prm.scale);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" int attn_bwd_workspace_size(int B, int H, int Nq, int Nk, int d, size_t* bytes) {
+  if (bytes == nullptr) return ATTN_ERR_NULL;
+  if (d != 64 && d != 128) return ATTN_ERR_HEAD_DIM;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1) return ATTN_ERR_SHAPE;
+  *bytes = bwd_workspace_bytes(static_cast<long long>(B) * H, Nq, d);
+  return ATTN_OK;
+}
+
+extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                        const float* lse, const void* dout, void* dq, void* dk, void* dv, int B,
+                        int H, int Nq, int Nk, int d, float scale, int causal, int dtype,
+                        void* workspace, size_t workspace_bytes, attn_stream_t stream) {
+  int st = check_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, dtype);
+  if (st != ATTN_OK) return st;
+  if (lse == nullptr || dout == nullptr || dq == nullptr || dk == nullptr || dv == nullptr)
+    return ATTN_ERR_NULL;
+  auto misaligned = [](const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) != 0; };
+  if (misaligned(dout) || misaligned(dq) || misaligned(dk) || misaligned(dv)) return ATTN_ERR_ALIGN;
+  const long long BH = static_cast<long long>(B) * H;
+  const int nk_tiles = ceil_div(Nk, BLOCK_N);
+  if (BH * nk_tiles >= (1LL << 31)) return ATTN_ERR_SHAPE;
+  if (workspace == nullptr || misaligned(workspace) ||
+      workspace_bytes < bwd_workspace_bytes(BH, Nq, d))
+    return ATTN_ERR_WORKSPACE;
+  int dev = -1;
+  DeviceInfo* info = nullptr;
+  st = current_device(&dev, &info);
+  if (st != ATTN_OK) return st;
+  const MapCache* maps = cached_maps(q, k, v, Nq, Nk, BH, d, dtype, dev);
+  if (maps == nullptr) return ATTN_ERR_CUDA;
+  BwdMapCache& dm = t_do_map;
+  if (dm.dout != dout || dm.Nq != Nq || dm.d != d || dm.dtype != dtype || dm.dev != dev ||
+      dm.BH != BH) {
+    dm.dout = nullptr;
+    if (!encode_map(&dm.m, dout, Nq, BH, d, dtype)) return ATTN_ERR_CUDA;
+    dm.dout = dout; dm.Nq = Nq; dm.d = d; dm.dtype = dtype; dm.dev = dev; dm.BH = BH;
+  }
+  attn_sm100::BwdParams prm;
+  const int nq_tiles = ceil_div(Nq, BLOCK_M);
+  const int nq_pad = nq_tiles * BLOCK_M;
+  char* ws = static_cast<char*>(workspace);
+  prm.dk = dk;
+  prm.dv = dv;
+  prm.dq_acc = reinterpret_cast<float*>(ws);
+  prm.lse2 = reinterpret_cast<const float*>(ws + static_cast<size_t>(BH) * Nq * d * 4);
+  prm.dsum = prm.lse2 + static_cast<size_t>(BH) * nq_pad;
+  prm.Nq = Nq;
+  prm.Nk = Nk;
+  prm.BH = static_cast<int>(BH);
+  prm.nq_tiles = nq_tiles;
+  prm.nk_tiles = nk_tiles;
+  prm.nq_pad = nq_pad;
+  prm.causal = causal ? 1 : 0;
+  prm.scale = scale;
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    return dtype == ATTN_BF16
+               ? bwd_launch<64, true>(*maps, dm.m, o, dout, lse, dq, prm, dev, info->sms, s)
+               : bwd_launch<64, false>(*maps, dm.m, o, dout, lse, dq, prm, dev, info->sms, s);
+  return dtype == ATTN_BF16
+             ? bwd_launch<128, true>(*maps, dm.m, o, dout, lse, dq, prm, dev, info->sms, s)
+             : bwd_launch<128, false>(*maps, dm.m, o, dout, lse, dq, prm, dev, info->sms, s);
+}
 
 // ---------------------------------------------------------------------------
 // Allocation-free entry point.

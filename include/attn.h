@@ -57,7 +57,8 @@ typedef enum {
   ATTN_ERR_ARCH = 7,           /* current device is not compute capability 10.0 (B200) */
   ATTN_ERR_CUDA = 8,           /* a CUDA runtime / driver call failed (no device, launch error) */
   ATTN_ERR_DEVICE_TIMEOUT = 9, /* a kernel gave up waiting (see attn_get_device_status) */
-  ATTN_ERR_SCRATCH_LIMIT = 10   /* attn_fwd_noalloc: the problem needs more than its fixed scratch */
+  ATTN_ERR_SCRATCH_LIMIT = 10,  /* attn_fwd_noalloc: the problem needs more than its fixed scratch */
+  ATTN_ERR_WORKSPACE = 11       /* attn_bwd: workspace NULL, smaller than required or not 16-byte aligned */
 } attn_status_t;
 
 /* Launch geometry for one call (see attn_plan). */
@@ -225,6 +226,43 @@ int attn_fwd_host(const void* q_host, const void* k_host, const void* v_host, vo
                   float* lse_host, void* q_dev, void* k_dev, void* v_dev, void* o_dev,
                   float* lse_dev, void* workspace, size_t workspace_bytes, int B, int H, int Nq,
                   int Nk, int d, float scale, int causal, int dtype, attn_stream_t stream);
+
+/*
+ * attn_bwd -- gradients of the forward: dq, dk, dv for an output gradient dout.
+ *
+ * The backward pass of training, with the softmax recomputed from the statistics the forward
+ * saved instead of being stored ("YOLOv12推理速度翻倍秘诀：Flash Attention加持" (0539edu.com),
+ * section 1; YOLO11 x FlashAttention-2 (kwkr.cn), sections 2.3 and 4.3).  For each (batch,
+ * head), with S = scale * Q K^T (masked as in attn_fwd) and P = exp(S - lse):
+ *   dV = P^T dO,  dS = P * (dO V^T - rowsum(dO * O)),  dQ = scale * dS K,  dK = scale * dS^T Q.
+ *
+ *   q, k, v    the forward's inputs (layouts of attn_fwd).
+ *   o, lse     the forward's outputs for exactly these inputs, scale and causal flag: o
+ *              [B, H, Nq, d] in `dtype`, lse [B, H, Nq] float32 (lse is required here).
+ *   dout       dL/dO, [B, H, Nq, d] in `dtype`.
+ *   dq, dk, dv outputs, shaped and typed like q, k, v (fully overwritten; rows a causal mask
+ *              hides from every query get zero gradients).
+ *   workspace  caller-owned device memory of at least attn_bwd_workspace_size bytes,
+ *              16-byte aligned; contents need not be initialised and are left undefined.
+ *
+ * Three kernels run in order on `stream`: a row pass (D = rowsum(dO * O), lse in base 2,
+ * zeroing an fp32 dQ accumulator in the workspace), the main pass (one CTA per 128-key tile
+ * and (batch, head): recomputed P, dS, and dK, dV accumulated in tensor memory, dQ added into
+ * the accumulator with atomic vector adds) and a pass converting dQ to `dtype`.  Because the
+ * dQ additions from different key tiles land in any order, dq can differ in the last bits
+ * between calls; dk and dv are deterministic.
+ *
+ * Errors: as attn_fwd for q, k, v, o, lse (NULL lse is ATTN_ERR_NULL) and for dout, dq, dk, dv
+ * (NULL, 16-byte alignment); ATTN_ERR_WORKSPACE for the workspace.  Nothing is enqueued on an
+ * argument error.  Nothing is allocated per call.
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             const void* dout, void* dq, void* dk, void* dv, int B, int H, int Nq, int Nk, int d,
+             float scale, int causal, int dtype, void* workspace, size_t workspace_bytes,
+             attn_stream_t stream);
+
+/* Workspace bytes attn_bwd needs for these sizes (host arithmetic only; no GPU needed). */
+int attn_bwd_workspace_size(int B, int H, int Nq, int Nk, int d, size_t* bytes);
 
 /*
  * attn_plan -- the launch geometry attn_fwd would use for these sizes on a GPU with

@@ -35,7 +35,7 @@ def test_header_declares_the_boundary():
     assert header_functions() == sorted([
         "attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_noalloc", "attn_fwd_host",
         "attn_fwd_stall_test", "attn_plan", "attn_get_device_status", "attn_strerror",
-        "attn_version"])
+        "attn_version", "attn_bwd", "attn_bwd_workspace_size"])
 
 
 def test_every_declared_symbol_is_exported():
@@ -55,7 +55,7 @@ def test_status_enum_matches_header():
 
 
 def test_strerror_and_version():
-    for code in range(11):
+    for code in range(12):
         assert A.attn_strerror(code) != "unknown status"
     assert A.attn_strerror(1234) == "unknown status"
     assert A.attn_version() == 100
@@ -190,3 +190,39 @@ def test_plan_errors(kw, code):
     with pytest.raises(A.AttnError) as e:
         A.attn_plan(*a.values())
     assert e.value.status == code
+
+
+# ------------------------------------------------------------------ backward arguments
+
+BWD = dict(q=0x10000, k=0x20000, v=0x30000, o=0x40000, lse=0x50000, do=0x60000, dq=0x70000,
+           dk=0x80000, dv=0x90000, B=1, H=2, Nq=400, Nk=300, d=64, scale=0.125, causal=0,
+           dtype=A.ATTN_FP16, ws=0xA0000, ws_bytes=1 << 30)
+
+
+def call_bwd(**kw):
+    a = dict(BWD)
+    a.update(kw)
+    return A.attn_bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["do"], a["dq"], a["dk"],
+                      a["dv"], a["B"], a["H"], a["Nq"], a["Nk"], a["d"], a["scale"], a["causal"],
+                      a["dtype"], a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(lse=None), 1), (dict(do=None), 1), (dict(dq=None), 1),
+    (dict(dk=None), 1), (dict(dv=None), 1),
+    (dict(dtype=3), 4), (dict(d=96), 3), (dict(Nq=0), 2), (dict(Nk=0), 2),
+    (dict(do=0x60002), 5), (dict(dq=0x70008), 5), (dict(dk=0x80004), 5), (dict(dv=0x90001), 5),
+    (dict(scale=0.0), 6),
+    (dict(ws=None), 11), (dict(ws=0xA0004), 11), (dict(ws_bytes=1000), 11),
+])
+def test_bwd_argument_errors(kw, code):
+    assert call_bwd(**kw) == code
+
+
+def test_bwd_workspace_size():
+    # fp32 dQ accumulator plus two padded per-row vectors
+    n = A.attn_bwd_workspace_size(2, 3, 200, 77, 64)
+    assert n == 2 * 3 * 200 * 64 * 4 + 2 * 2 * 3 * 256 * 4
+    assert A.attn_bwd_workspace_size(1, 1, 128, 1, 128) == 128 * 128 * 4 + 2 * 128 * 4
+    with pytest.raises(A.AttnError):
+        A.attn_bwd_workspace_size(1, 1, 128, 1, 80)
