@@ -1,4 +1,4 @@
-"""CPU float64 oracle for the exact attention forward and its gradients.
+"""CPU float64 oracle for the exact attention forward, its gradients and its block.
 
 TEST INFRASTRUCTURE ONLY: imported by ``tests/``, ``__graft_entry__.smoke()``
 and the CPU-baseline leg of ``bench.py``.  The CUDA path never imports it.
@@ -12,3 +12,4 @@ from .backward import (  # noqa: F401
     attention_backward_f64, grad_k, grad_p, grad_q, grad_scores, grad_v, recompute_probs,
     row_dot,
 )
+from .block import attention_block_f64, linear, merge_heads, split_qkv  # noqa: F401
