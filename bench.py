@@ -395,11 +395,13 @@ def main():
 
     per_workload = None
     backward = None
+    blocks = None
     cpu = None
     if rank == 0 and world == 1 and not args.no_per_workload:
         per_workload = context_timings(attn, torch, dev, peaks, steps=args.steps,
                                        warmup=args.warmup, device_index=local)
         backward = backward_timings(attn, torch, dev, peaks, warmup=args.warmup)
+        blocks = block_timings(attn, torch, dev, peaks, warmup=args.warmup)
     if rank == 0:
         flops, dt, done = time_oracle_sample(w, q, k, v, budget_s=args.cpu_budget)
         cpu = {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": blas_threads() or cpu_cores(),
@@ -432,6 +434,8 @@ def main():
             line["per_workload"] = per_workload
         if backward is not None:
             line["backward"] = backward
+        if blocks is not None:
+            line["block"] = blocks
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -477,6 +481,67 @@ def backward_timings(attn, torch, dev, peaks, steps=20, warmup=3):
                        "frac": round(tf / peaks["bf16_tflops"], 4), "bound": "tensor",
                        "launches": 3}
         del q, k, v, do, o, lse, ws, grads
+        torch.cuda.empty_cache()
+    return out
+
+
+BLOCK_CONFIGS = [
+    # name, B, N, H, d, dtype, causal: the attention block around two of the workloads
+    ("yolo_neck_40x40_b16_block", 16, 1600, 4, 64, "fp16", False),
+    ("llm_causal_2048_block", 32, 2048, 16, 64, "fp16", True),
+]
+
+
+def block_timings(attn, torch, dev, peaks, steps=20, warmup=3):
+    """µs per attn_block_fwd call (qkv GEMM, attention, output GEMM; L2 flushed before each
+    call) and the time of each of its three kernels alone."""
+    from seeded_inputs import make_block_inputs
+    out = {}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    for name, B, N, H, d, dtype, causal in BLOCK_CONFIGS:
+        C = H * d
+        x, w_qkv, b_qkv, w_o, b_o = (t.to(dev) if t is not None else None
+                                     for t in make_block_inputs(B, N, H, d, C, dtype, seed=7))
+        q, k, v, o = (torch.empty((B, H, N, d), dtype=x.dtype, device=dev) for _ in range(4))
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        y = torch.empty_like(x)
+        code = attn.ATTN_BF16 if dtype == "bf16" else attn.ATTN_FP16
+        sh = torch.cuda.current_stream().cuda_stream
+        calls = {
+            "block": lambda: attn.attn_block_fwd(
+                x.data_ptr(), w_qkv.data_ptr(), None, w_o.data_ptr(), b_o.data_ptr(),
+                q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                y.data_ptr(), B, N, H, d, C, 1.0 / math.sqrt(d), causal, code, sh),
+            "qkv_proj": lambda: attn.attn_qkv_proj(x.data_ptr(), w_qkv.data_ptr(), None,
+                                                   q.data_ptr(), k.data_ptr(), v.data_ptr(), B,
+                                                   N, H, d, code, sh),
+            "attention": lambda: attn.attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                               o.data_ptr(), lse.data_ptr(), B, H, N, N, d,
+                                               1.0 / math.sqrt(d), causal, code, sh),
+            "out_proj": lambda: attn.attn_out_proj(o.data_ptr(), w_o.data_ptr(), b_o.data_ptr(),
+                                                   y.data_ptr(), B, N, H, d, C, code, sh),
+        }
+        res = {"B": B, "N": N, "H": H, "d": d, "C": C, "dtype": dtype, "causal": causal}
+        for part, fn in calls.items():
+            for _ in range(max(3, warmup)):
+                assert fn() == 0
+            times = []
+            for _ in range(steps):
+                flush.zero_()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                assert fn() == 0
+                e1.record()
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1) * 1e3)
+            res[part + "_us"] = round(percentiles(times)["median"], 2)
+        gemm_flops = 2.0 * B * N * C * 3 * C + 2.0 * B * N * C * C
+        attn_flops = 4.0 * B * H * N * N * d / (2.0 if causal else 1.0)
+        res["tflops"] = round((gemm_flops + attn_flops) / (res["block_us"] * 1e-6) / 1e12, 2)
+        res["qkv_proj_tflops"] = round(2.0 * B * N * C * 3 * C / (res["qkv_proj_us"] * 1e-6) / 1e12, 2)
+        res["out_proj_tflops"] = round(2.0 * B * N * C * C / (res["out_proj_us"] * 1e-6) / 1e12, 2)
+        out[name] = res
+        del x, w_qkv, w_o, b_o, q, k, v, o, lse, y
         torch.cuda.empty_cache()
     return out
 

@@ -23,6 +23,7 @@ __all__ = [
     "attn_plan", "attn_get_device_status", "attn_strerror", "attn_version", "forward",
     "forward_host", "STATUS_NAMES", "attn_fwd_ws", "attn_workspace_size", "workspace_for",
     "attn_fwd_noalloc", "attn_bwd", "attn_bwd_workspace_size", "backward",
+    "attn_qkv_proj", "attn_out_proj", "attn_block_fwd", "qkv_proj", "out_proj", "block_forward",
 ]
 
 ATTN_FP16 = 0
@@ -91,6 +92,12 @@ def lib() -> ctypes.CDLL:
         L.attn_bwd.restype = i
         L.attn_bwd_workspace_size.argtypes = [i, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
         L.attn_bwd_workspace_size.restype = i
+        L.attn_qkv_proj.argtypes = [vp] * 6 + [i, i, i, i, i, vp]
+        L.attn_qkv_proj.restype = i
+        L.attn_out_proj.argtypes = [vp] * 4 + [i, i, i, i, i, i, vp]
+        L.attn_out_proj.restype = i
+        L.attn_block_fwd.argtypes = [vp] * 11 + [i, i, i, i, i, f, i, i, vp]
+        L.attn_block_fwd.restype = i
         L.attn_plan.argtypes = [i, i, i, i, i, i, i, ctypes.POINTER(_Plan)]
         L.attn_plan.restype = i
         L.attn_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
@@ -147,6 +154,23 @@ def attn_bwd_workspace_size(B, H, Nq, Nk, d) -> int:
     if st != 0:
         raise AttnError(st, "attn_bwd_workspace_size")
     return n.value
+
+
+def attn_qkv_proj(x, w_qkv, b_qkv, q, k, v, B, N, H, d, dtype, stream) -> int:
+    """Raw ``attn_qkv_proj``: pointers and the stream handle as Python ints."""
+    return lib().attn_qkv_proj(x, w_qkv, b_qkv, q, k, v, B, N, H, d, dtype, stream)
+
+
+def attn_out_proj(o, w_o, b_o, y, B, N, H, d, C_out, dtype, stream) -> int:
+    """Raw ``attn_out_proj``."""
+    return lib().attn_out_proj(o, w_o, b_o, y, B, N, H, d, C_out, dtype, stream)
+
+
+def attn_block_fwd(x, w_qkv, b_qkv, w_o, b_o, q, k, v, o, lse, y, B, N, H, d, C_out, scale,
+                   causal, dtype, stream) -> int:
+    """Raw ``attn_block_fwd``."""
+    return lib().attn_block_fwd(x, w_qkv, b_qkv, w_o, b_o, q, k, v, o, lse, y, B, N, H, d, C_out,
+                                float(scale), int(causal), dtype, stream)
 
 
 def attn_workspace_size(B, H, Nq, Nk, d, causal) -> int:
@@ -308,3 +332,57 @@ def backward(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
     if st != 0:
         raise AttnError(st, "attn_bwd")
     return dq, dk, dv
+
+
+def _ptr(t):
+    return t.data_ptr() if t is not None else None
+
+
+def qkv_proj(x, w_qkv, b_qkv, H: int, stream=None, out=None):
+    """q, k, v [B, H, N, d] = the head split of x W_qkv^T (+ b_qkv), x [B, N, C]."""
+    import torch
+    B, N, C = x.shape
+    d = C // H
+    if d * H != C:
+        raise ValueError("C must be H * d")
+    q, k, v = out if out is not None else tuple(
+        torch.empty((B, H, N, d), dtype=x.dtype, device=x.device) for _ in range(3))
+    st = attn_qkv_proj(x.data_ptr(), w_qkv.data_ptr(), _ptr(b_qkv), q.data_ptr(), k.data_ptr(),
+                       v.data_ptr(), B, N, H, d, _dtype_code(x), _stream_handle(stream))
+    if st != 0:
+        raise AttnError(st, "attn_qkv_proj")
+    return q, k, v
+
+
+def out_proj(o, w_o, b_o, stream=None, out=None):
+    """y [B, N, C_out] = o' W_o^T (+ b_o), o' the [B, N, H d] view of o [B, H, N, d]."""
+    import torch
+    B, H, N, d = o.shape
+    C_out = w_o.shape[0]
+    y = out if out is not None else torch.empty((B, N, C_out), dtype=o.dtype, device=o.device)
+    st = attn_out_proj(o.data_ptr(), w_o.data_ptr(), _ptr(b_o), y.data_ptr(), B, N, H, d, C_out,
+                       _dtype_code(o), _stream_handle(stream))
+    if st != 0:
+        raise AttnError(st, "attn_out_proj")
+    return y
+
+
+def block_forward(x, w_qkv, b_qkv, w_o, b_o, H: int, causal: bool = False, scale=None,
+                  stream=None):
+    """The attention block: returns (y, q, k, v, o, lse)."""
+    import torch
+    B, N, C = x.shape
+    d = C // H
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    q, k, v, o = (torch.empty((B, H, N, d), dtype=x.dtype, device=x.device) for _ in range(4))
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=x.device)
+    C_out = w_o.shape[0]
+    y = torch.empty((B, N, C_out), dtype=x.dtype, device=x.device)
+    st = attn_block_fwd(x.data_ptr(), w_qkv.data_ptr(), _ptr(b_qkv), w_o.data_ptr(), _ptr(b_o),
+                        q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                        y.data_ptr(), B, N, H, d, C_out, scale, causal, _dtype_code(x),
+                        _stream_handle(stream))
+    if st != 0:
+        raise AttnError(st, "attn_block_fwd")
+    return y, q, k, v, o, lse

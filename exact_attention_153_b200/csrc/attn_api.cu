@@ -18,6 +18,7 @@
 #include "attn.h"
 #include "attn_bwd_sm100.cuh"
 #include "attn_fwd_sm100.cuh"
+#include "proj_gemm_sm100.cuh"
 
 namespace {
 
@@ -718,6 +719,187 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
   return dtype == ATTN_BF16
              ? bwd_launch<128, true>(*maps, dm.m, o, dout, lse, dq, prm, dev, info->sms, s)
              : bwd_launch<128, false>(*maps, dm.m, o, dout, lse, dq, prm, dev, info->sms, s);
+}
+
+// ---------------------------------------------------------------------------
+// Projections of the attention block (QKV in, output out), fused with the
+// [B, H, N, d] layout of the attention.
+// ---------------------------------------------------------------------------
+namespace {
+
+// Tiled map of a 16-bit tensor of `rank` dims (innermost first), strides in
+// bytes for dims 1.., boxes of 64 x 128 (x 1 ...) with the 128-byte swizzle.
+bool encode_tiled(CUtensorMap* map, const void* ptr, int rank, const cuuint64_t* dims,
+                  const cuuint64_t* strides, int dtype) {
+  EncodeTiledFn enc = encode_fn();
+  if (enc == nullptr) return false;
+  const cuuint32_t box[5] = {64, 128, 1, 1, 1};
+  const cuuint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+  return enc(map, dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+             rank, const_cast<void*>(ptr), dims, strides, box, elem_strides,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// [rows, cols] row-major 16-bit matrix as the 3-D map (cols, rows, 1).
+bool encode_matrix(CUtensorMap* map, const void* ptr, long long rows, long long cols, int dtype) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), 1};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2,
+                                 static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols) * 2};
+  return encode_tiled(map, ptr, 3, dims, strides, dtype);
+}
+
+std::atomic<bool> g_proj_attr[kMaxDevices][2][2];  // [dev][bf16][mode]
+
+template <bool BF16, int MODE>
+int proj_launch(const CUtensorMap& ma, const CUtensorMap& mb, const attn_sm100::ProjParams& prm,
+                int m_tiles_total, int dev, cudaStream_t stream) {
+  auto kernel = attn_sm100::proj_gemm_kernel<BF16, MODE>;
+  constexpr int smem = attn_sm100::ProjSmem::BYTES;
+  std::atomic<bool>& attr = g_proj_attr[dev][BF16][MODE];
+  if (!attr.load(std::memory_order_acquire)) {
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    if (!attr.load(std::memory_order_relaxed)) {
+      if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+          cudaSuccess) {
+        cudaGetLastError();
+        return ATTN_ERR_CUDA;
+      }
+      attr.store(true, std::memory_order_release);
+    }
+  }
+  const dim3 grid(static_cast<unsigned int>(ceil_div(prm.N_out, 128)),
+                  static_cast<unsigned int>(m_tiles_total));
+  kernel<<<grid, attn_sm100::PROJ_THREADS, smem, stream>>>(ma, mb, prm);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+bool aligned16(const void* ptr) { return (reinterpret_cast<uintptr_t>(ptr) & 15) == 0; }
+
+int check_proj_shape(int B, int N, int H, int d, int dtype) {
+  if (dtype != ATTN_FP16 && dtype != ATTN_BF16) return ATTN_ERR_DTYPE;
+  if (d != 64 && d != 128) return ATTN_ERR_HEAD_DIM;
+  if (B < 1 || N < 1 || H < 1) return ATTN_ERR_SHAPE;
+  const long long rows = static_cast<long long>(B) * N;
+  if (rows >= (1LL << 31) / 2 || static_cast<long long>(H) * d * 3 >= (1LL << 30) ||
+      (rows + 127) / 128 >= 65535)
+    return ATTN_ERR_SHAPE;
+  return ATTN_OK;
+}
+
+int qkv_proj_impl(const void* x, const void* w_qkv, const float* b_qkv, void* q, void* k, void* v,
+                  int B, int N, int H, int d, int dtype, cudaStream_t s) {
+  int st = check_proj_shape(B, N, H, d, dtype);
+  if (st != ATTN_OK) return st;
+  if (x == nullptr || w_qkv == nullptr || q == nullptr || k == nullptr || v == nullptr)
+    return ATTN_ERR_NULL;
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+      (b_qkv != nullptr && (reinterpret_cast<uintptr_t>(b_qkv) & 3) != 0))
+    return ATTN_ERR_ALIGN;
+  int dev = -1;
+  DeviceInfo* info = nullptr;
+  st = current_device(&dev, &info);
+  if (st != ATTN_OK) return st;
+  const int C = H * d;
+  const long long M = static_cast<long long>(B) * N;
+  CUtensorMap ma, mb;
+  if (!encode_matrix(&ma, x, M, C, dtype) || !encode_matrix(&mb, w_qkv, 3LL * C, C, dtype))
+    return ATTN_ERR_CUDA;
+  attn_sm100::ProjParams prm;
+  prm.bias = b_qkv;
+  prm.out0 = q;
+  prm.out1 = k;
+  prm.out2 = v;
+  prm.B = B;
+  prm.N = N;
+  prm.K = C;
+  prm.N_out = 3 * C;
+  prm.H = H;
+  prm.d = d;
+  prm.m_tiles = static_cast<int>((M + 127) / 128);
+  return dtype == ATTN_BF16
+             ? proj_launch<true, attn_sm100::PROJ_QKV>(ma, mb, prm, prm.m_tiles, dev, s)
+             : proj_launch<false, attn_sm100::PROJ_QKV>(ma, mb, prm, prm.m_tiles, dev, s);
+}
+
+int out_proj_impl(const void* o, const void* w_o, const float* b_o, void* y, int B, int N, int H,
+                  int d, int C_out, int dtype, cudaStream_t s) {
+  int st = check_proj_shape(B, N, H, d, dtype);
+  if (st != ATTN_OK) return st;
+  if (C_out < 8 || C_out % 8 != 0 || C_out >= (1 << 30)) return ATTN_ERR_SHAPE;
+  if (static_cast<long long>(B) * ceil_div(N, 128) >= 65535) return ATTN_ERR_SHAPE;  // grid rows
+  if (o == nullptr || w_o == nullptr || y == nullptr) return ATTN_ERR_NULL;
+  if (!aligned16(o) || !aligned16(w_o) || !aligned16(y) ||
+      (b_o != nullptr && (reinterpret_cast<uintptr_t>(b_o) & 3) != 0))
+    return ATTN_ERR_ALIGN;
+  int dev = -1;
+  DeviceInfo* info = nullptr;
+  st = current_device(&dev, &info);
+  if (st != ATTN_OK) return st;
+  const int C = H * d;
+  CUtensorMap ma, mb;
+  // o [B, H, N, d] as the 4-D map (d, N, H, B): box (64, 128, 1, 1) is 128 rows of
+  // o' = [B N, H d] over 64 of its columns, inside one head
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(H), static_cast<cuuint64_t>(B)};
+  const cuuint64_t strides[3] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(N) * d * 2,
+                                 static_cast<cuuint64_t>(H) * N * d * 2};
+  if (!encode_tiled(&ma, o, 4, dims, strides, dtype) || !encode_matrix(&mb, w_o, C_out, C, dtype))
+    return ATTN_ERR_CUDA;
+  attn_sm100::ProjParams prm;
+  prm.bias = b_o;
+  prm.out0 = y;
+  prm.out1 = prm.out2 = nullptr;
+  prm.B = B;
+  prm.N = N;
+  prm.K = C;
+  prm.N_out = C_out;
+  prm.H = H;
+  prm.d = d;
+  prm.m_tiles = ceil_div(N, 128);
+  const int m_total = B * prm.m_tiles;
+  return dtype == ATTN_BF16 ? proj_launch<true, attn_sm100::PROJ_OUT>(ma, mb, prm, m_total, dev, s)
+                            : proj_launch<false, attn_sm100::PROJ_OUT>(ma, mb, prm, m_total, dev, s);
+}
+
+}  // namespace
+
+extern "C" int attn_qkv_proj(const void* x, const void* w_qkv, const float* b_qkv, void* q,
+                             void* k, void* v, int B, int N, int H, int d, int dtype,
+                             attn_stream_t stream) {
+  return qkv_proj_impl(x, w_qkv, b_qkv, q, k, v, B, N, H, d, dtype,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int attn_out_proj(const void* o, const void* w_o, const float* b_o, void* y, int B,
+                             int N, int H, int d, int C_out, int dtype, attn_stream_t stream) {
+  return out_proj_impl(o, w_o, b_o, y, B, N, H, d, C_out, dtype,
+                       reinterpret_cast<cudaStream_t>(stream));
+}
+
+extern "C" int attn_block_fwd(const void* x, const void* w_qkv, const float* b_qkv,
+                              const void* w_o, const float* b_o, void* q, void* k, void* v,
+                              void* o, float* lse, void* y, int B, int N, int H, int d,
+                              int C_out, float scale, int causal, int dtype,
+                              attn_stream_t stream) {
+  // every argument is checked before the first launch
+  int st = check_proj_shape(B, N, H, d, dtype);
+  if (st != ATTN_OK) return st;
+  if (C_out < 8 || C_out % 8 != 0) return ATTN_ERR_SHAPE;
+  if (x == nullptr || w_qkv == nullptr || w_o == nullptr || y == nullptr) return ATTN_ERR_NULL;
+  st = check_args(q, k, v, o, lse, B, H, N, N, d, scale, dtype);
+  if (st != ATTN_OK) return st;
+  if (!aligned16(x) || !aligned16(w_qkv) || !aligned16(w_o) || !aligned16(y) ||
+      (b_qkv != nullptr && (reinterpret_cast<uintptr_t>(b_qkv) & 3) != 0) ||
+      (b_o != nullptr && (reinterpret_cast<uintptr_t>(b_o) & 3) != 0))
+    return ATTN_ERR_ALIGN;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  st = qkv_proj_impl(x, w_qkv, b_qkv, q, k, v, B, N, H, d, dtype, s);
+  if (st != ATTN_OK) return st;
+  st = fwd_impl(q, k, v, o, lse, B, H, N, N, d, scale, causal, dtype, nullptr, 0, stream);
+  if (st != ATTN_OK) return st;
+  return out_proj_impl(o, w_o, b_o, y, B, N, H, d, C_out, dtype, s);
 }
 
 // ---------------------------------------------------------------------------

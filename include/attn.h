@@ -265,6 +265,45 @@ int attn_bwd(const void* q, const void* k, const void* v, const void* o, const f
 int attn_bwd_workspace_size(int B, int H, int Nq, int Nk, int d, size_t* bytes);
 
 /*
+ * attn_qkv_proj -- the qkv projection of the attention block, written in the attention layout.
+ *
+ * [q | k | v] = x W_qkv^T (+ b_qkv) for x [B, N, C] with C = H * d, W_qkv [3 C, C] (an
+ * nn.Linear(C, 3 C) weight) and b_qkv [3 C] float32 or NULL (the page's qkv Linear has no
+ * bias).  Column c of the product goes to tensor c / C (q, k, v), head (c % C) / d, element
+ * c % d -- the reshape to [B, N, 3, H, d], unbind and transpose of the YOLO11 x
+ * FlashAttention-2 page (kwkr.cn), section 2.2 -- so q, k, v come out as [B, H, N, d]
+ * contiguous, ready for attn_fwd, with no reshape pass.  One tcgen05 GEMM (fp32 accumulation,
+ * one rounding to `dtype`).  x, W_qkv, q, k, v 16-byte aligned; b_qkv 4-byte aligned.  Errors:
+ * ATTN_ERR_NULL, ATTN_ERR_DTYPE, ATTN_ERR_HEAD_DIM (d not 64 / 128), ATTN_ERR_SHAPE,
+ * ATTN_ERR_ALIGN, ATTN_ERR_ARCH, ATTN_ERR_CUDA; nothing is enqueued on an argument error.
+ */
+int attn_qkv_proj(const void* x, const void* w_qkv, const float* b_qkv, void* q, void* k,
+                  void* v, int B, int N, int H, int d, int dtype, attn_stream_t stream);
+
+/*
+ * attn_out_proj -- the output projection, reading the attention output in its own layout.
+ *
+ * y = o' W_o^T (+ b_o) where o' [B, N, H d] is o [B, H, N, d] transposed back (the page's
+ * o.transpose(1, 2).reshape(B, N, C)), W_o [C_out, H d] and b_o [C_out] float32 or NULL; y is
+ * [B, N, C_out] in `dtype`.  The GEMM's first operand is loaded from o through a 4-D tensor
+ * map, so the transpose is never written out.  C_out must be a multiple of 8.  o, W_o, y
+ * 16-byte aligned.  Errors as attn_qkv_proj.
+ */
+int attn_out_proj(const void* o, const void* w_o, const float* b_o, void* y, int B, int N, int H,
+                  int d, int C_out, int dtype, attn_stream_t stream);
+
+/*
+ * attn_block_fwd -- the whole attention block: attn_qkv_proj, attn_fwd (Nq = Nk = N), then
+ * attn_out_proj, enqueued in that order on `stream` after every argument has been checked.
+ * q, k, v, o [B, H, N, d] and lse [B, H, N] (or NULL) are caller-owned intermediates and keep
+ * their values.  Errors as the three calls.
+ */
+int attn_block_fwd(const void* x, const void* w_qkv, const float* b_qkv, const void* w_o,
+                   const float* b_o, void* q, void* k, void* v, void* o, float* lse, void* y,
+                   int B, int N, int H, int d, int C_out, float scale, int causal, int dtype,
+                   attn_stream_t stream);
+
+/*
  * attn_plan -- the launch geometry attn_fwd would use for these sizes on a GPU with
  * `num_sms` SMs (pure host arithmetic; needs no GPU).  Returns ATTN_ERR_SHAPE /
  * ATTN_ERR_HEAD_DIM / ATTN_ERR_NULL on bad arguments, else ATTN_OK with *out filled.

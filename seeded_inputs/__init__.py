@@ -30,7 +30,8 @@ from dataclasses import dataclass, field
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "workload", "make_qkv", "dtype_of"]
+__all__ = ["Workload", "WORKLOADS", "workload", "make_qkv", "dtype_of", "make_grad_out",
+           "make_workload_qkv", "make_block_inputs"]
 
 _DTYPES = {"fp16": torch.float16, "bf16": torch.bfloat16}
 
@@ -137,3 +138,21 @@ def make_grad_out(B: int, H: int, Nq: int, dv: int, dtype: str, seed: int):
 def make_workload_qkv(w: Workload):
     """Inputs of a named workload."""
     return make_qkv(w.B, w.H, w.Nq, w.Nk, w.d, w.dtype, w.seed, w.qk_scale)
+
+
+def make_block_inputs(B: int, N: int, H: int, d: int, C_out: int, dtype: str, seed: int,
+                      qkv_bias: bool = False):
+    """Seeded input and weights of an attention block: x [B, N, C] N(0,1), W_qkv [3C, C] and
+    W_o [C_out, C] N(0, 1/C) (the scale of a default-initialised Linear), b_o [C_out] fp32
+    N(0, 0.1^2), and b_qkv [3C] fp32 likewise when ``qkv_bias`` (the page's qkv Linear has
+    none).  Returns (x, w_qkv, b_qkv or None, w_o, b_o)."""
+    C = H * d
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed) + 104729)
+    t = dtype_of(dtype)
+    x = torch.randn((B, N, C), generator=g, dtype=torch.float32).to(t).contiguous()
+    w_qkv = (torch.randn((3 * C, C), generator=g, dtype=torch.float32) / C ** 0.5).to(t).contiguous()
+    w_o = (torch.randn((C_out, C), generator=g, dtype=torch.float32) / C ** 0.5).to(t).contiguous()
+    b_o = 0.1 * torch.randn((C_out,), generator=g, dtype=torch.float32)
+    b_qkv = 0.1 * torch.randn((3 * C,), generator=g, dtype=torch.float32) if qkv_bias else None
+    return x, w_qkv, b_qkv, w_o, b_o

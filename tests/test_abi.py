@@ -35,7 +35,8 @@ def test_header_declares_the_boundary():
     assert header_functions() == sorted([
         "attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_noalloc", "attn_fwd_host",
         "attn_fwd_stall_test", "attn_plan", "attn_get_device_status", "attn_strerror",
-        "attn_version", "attn_bwd", "attn_bwd_workspace_size"])
+        "attn_version", "attn_bwd", "attn_bwd_workspace_size", "attn_qkv_proj", "attn_out_proj",
+        "attn_block_fwd"])
 
 
 def test_every_declared_symbol_is_exported():
@@ -226,3 +227,27 @@ def test_bwd_workspace_size():
     assert A.attn_bwd_workspace_size(1, 1, 128, 1, 128) == 128 * 128 * 4 + 2 * 128 * 4
     with pytest.raises(A.AttnError):
         A.attn_bwd_workspace_size(1, 1, 128, 1, 80)
+
+
+# ------------------------------------------------------------------ projection arguments
+
+def test_proj_argument_errors():
+    good = dict(x=0x10000, w=0x20000, b=None, q=0x30000, k=0x40000, v=0x50000)
+    def qkv(**kw):
+        a = dict(good, B=1, N=100, H=2, d=64, dtype=A.ATTN_FP16)
+        a.update(kw)
+        return A.attn_qkv_proj(a["x"], a["w"], a["b"], a["q"], a["k"], a["v"], a["B"], a["N"],
+                               a["H"], a["d"], a["dtype"], None)
+    assert qkv(x=None) == 1 and qkv(v=None) == 1
+    assert qkv(dtype=5) == 4 and qkv(d=32) == 3 and qkv(N=0) == 2 and qkv(H=0) == 2
+    assert qkv(x=0x10008) == 5 and qkv(b=0x60002) == 5
+    def outp(**kw):
+        a = dict(o=0x10000, w=0x20000, b=None, y=0x30000, B=1, N=100, H=2, d=64, C_out=128,
+                 dtype=A.ATTN_BF16)
+        a.update(kw)
+        return A.attn_out_proj(a["o"], a["w"], a["b"], a["y"], a["B"], a["N"], a["H"], a["d"],
+                               a["C_out"], a["dtype"], None)
+    assert outp(y=None) == 1 and outp(C_out=100) == 2 and outp(C_out=0) == 2
+    assert outp(o=0x10004) == 5 and outp(d=100) == 3
+    assert A.attn_block_fwd(0x10000, 0x20000, None, 0x30000, None, 0x40000, 0x50000, 0x60000,
+                            0x70000, None, 0x80000, 1, 64, 2, 64, 128, 0.0, 0, 0, None) == 6
