@@ -60,7 +60,8 @@ class _Plan(ctypes.Structure):
                 ("grid", ctypes.c_int), ("block", ctypes.c_int), ("smem_bytes", ctypes.c_int),
                 ("stages", ctypes.c_int), ("qk_tile_products", ctypes.c_longlong),
                 ("split", ctypes.c_int), ("split_grid", ctypes.c_int),
-                ("split_units", ctypes.c_int), ("workspace_bytes", ctypes.c_longlong)]
+                ("split_units", ctypes.c_int), ("workspace_bytes", ctypes.c_longlong),
+                ("split_steps", ctypes.c_longlong)]
 
 
 def lib() -> ctypes.CDLL:

@@ -91,17 +91,20 @@ int check_args(const void* q, const void* k, const void* v, const void* o, const
 // (the last piece reads every other piece's O back).  The cost, in key-tile
 // steps, was fitted to split and unit timings of small problems on B200:
 // about 3.5 + 0.56 per piece at d = 64 and 2.5 + 1.03 per piece at d = 128.
-bool split_pays(long long units, int kv_tiles, long long total_steps, int num_sms, int causal,
-                int d) {
-  if (causal || total_steps < 2) return false;
+// `unit_steps`: key-tile steps of the largest unit-mode unit (nk; under the
+// causal mask a heavy query pair plus its light mirror); `piece_steps`: the
+// steps of the largest split-mode unit (one query pair).
+bool split_pays(long long units, long long unit_steps, long long total_steps,
+                long long piece_steps, int num_sms, int d) {
+  if (total_steps < 2) return false;
   const long long grid = units < num_sms ? units : num_sms;
   const long long waves = (units + grid - 1) / grid;
   const double eff = static_cast<double>(units) / static_cast<double>(grid * waves);
   if (eff >= 0.9 && units >= num_sms) return false;
-  const long long steps_unit = waves * kv_tiles;
+  const long long steps_unit = waves * unit_steps;
   const long long grid_s = total_steps < num_sms ? total_steps : num_sms;
   const long long steps_split = (total_steps + grid_s - 1) / grid_s;
-  const long long pieces = (static_cast<long long>(kv_tiles) * grid_s + total_steps - 1) / total_steps;
+  const long long pieces = (piece_steps * grid_s + total_steps - 1) / total_steps;
   const double cost = d == 64 ? 3.5 + 0.56 * pieces : 2.5 + 1.03 * pieces;
   return static_cast<double>(steps_unit - steps_split) > cost;
 }
@@ -109,6 +112,15 @@ bool split_pays(long long units, int kv_tiles, long long total_steps, int num_sm
 size_t split_workspace_bytes(int grid, int d, long long units) {
   const size_t rows = static_cast<size_t>(grid) * 2 * 2 * BLOCK_M;
   return rows * d * sizeof(float) + rows * sizeof(float) + static_cast<size_t>(units) * 4 + 16;
+}
+
+// Key-tile steps of query pair qp in split mode: query tile i sees min(nk, i + 1)
+// key tiles under the top-left causal mask, so the pair needs those of its
+// last tile; without the mask, nk.
+long long split_pair_steps(int qp, int q_tiles, int kv_tiles, int causal) {
+  if (!causal) return kv_tiles;
+  const int last_tile = (2 * qp + 1 < q_tiles) ? 2 * qp + 1 : 2 * qp;
+  return last_tile + 1 < kv_tiles ? last_tile + 1 : kv_tiles;
 }
 
 void fill_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, attn_plan_t* out) {
@@ -145,12 +157,29 @@ void fill_plan(int B, int H, int Nq, int Nk, int d, int causal, int num_sms, att
     }
   }
   out->qk_tile_products = per_head * B * H;
-  // split mode keeps plain units (one (batch, head) each): q_pairs per head
+  // split mode keeps plain units (one (batch, head) and query pair each)
   const long long split_units = BH * q_pairs;
-  const long long total_steps = split_units * kv_tiles;
-  out->split = split_pays(units, kv_tiles, total_steps, num_sms, causal, d) ? 1 : 0;
+  long long steps_per_head = 0, piece_steps = 0, unit_steps = 0;
+  for (int qp = 0; qp < q_pairs; ++qp) {
+    const long long s = split_pair_steps(qp, q_tiles, kv_tiles, causal);
+    steps_per_head += s;
+    piece_steps = s > piece_steps ? s : piece_steps;
+  }
+  if (causal) {  // a unit-mode unit streams a heavy pair and its light mirror
+    for (int b = 0; b < units_per_head; ++b) {
+      const int heavy = q_pairs - 1 - b;
+      const long long s = split_pair_steps(heavy, q_tiles, kv_tiles, 1) +
+                          (heavy != b ? split_pair_steps(b, q_tiles, kv_tiles, 1) : 0);
+      unit_steps = s > unit_steps ? s : unit_steps;
+    }
+  } else {
+    unit_steps = kv_tiles;
+  }
+  const long long total_steps = BH * steps_per_head;
+  out->split = split_pays(units, unit_steps, total_steps, piece_steps, num_sms, d) ? 1 : 0;
   out->split_grid = static_cast<int>(total_steps < num_sms ? total_steps : num_sms);
   out->split_units = static_cast<int>(split_units);
+  out->split_steps = total_steps;
   out->workspace_bytes =
       out->split ? static_cast<long long>(split_workspace_bytes(out->split_grid, d, split_units)) : 0;
 }
@@ -307,6 +336,8 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   prm.split = 0;
   prm.total_steps = 0;
+  prm.num_q_tiles = plan.num_q_tiles;
+  prm.steps_per_head = plan.split_steps / BH;
   prm.ws_o = nullptr;
   prm.ws_lse = nullptr;
   prm.ws_count = nullptr;
@@ -325,7 +356,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
     prm.units_per_head = plan.num_q_pairs;
     prm.num_units = plan.split_units;
     prm.dual_base = -1;
-    prm.total_steps = static_cast<long long>(plan.split_units) * plan.num_kv_tiles;
+    prm.total_steps = plan.split_steps;
     prm.ws_o = reinterpret_cast<float*>(ws);
     prm.ws_lse = reinterpret_cast<float*>(ws + rows * d * sizeof(float));
     // the piece counters start at zero (the caller zero-fills a new

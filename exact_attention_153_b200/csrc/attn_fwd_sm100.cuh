@@ -126,13 +126,17 @@ struct FwdParams {
   int last_q0;
   int causal;
   float scale_log2; // scale * log2(e)
-  // Split mode (non-causal only).  The units' key tiles are flattened into
-  // total_steps = num_units * num_kv_tiles steps and CTA c takes steps
+  // Split mode.  Every unit is one query pair of one (batch, head); its key
+  // tiles are flattened into total_steps = B H * steps_per_head steps (a
+  // pair needs num_kv_tiles of them, or under the causal mask only the tiles
+  // its later query tile sees) and CTA c takes steps
   // [c * total_steps / grid, (c + 1) * total_steps / grid), so every CTA does
   // the same work however the units divide.  A unit cut by a range boundary
   // is computed in pieces; each piece leaves its normalised O and lse in the
   // caller's workspace and the last piece to finish merges them.
   int split;
+  int num_q_tiles;         // ceil(Nq / 128)
+  long long steps_per_head;
   long long total_steps;
   float* ws_o;           // [grid][2 slots][2 tiles][128 rows][D]
   float* ws_lse;         // [grid][2 slots][2 tiles][128 rows]
@@ -221,7 +225,9 @@ __device__ __forceinline__ int unit_items(const FwdParams& p, int u) {
   return (b != p.num_q_pairs - 1 - b) ? 2 : 1;
 }
 
-template <bool DUAL>
+// PLAIN: unit b of a head is query pair b (split mode), without the causal
+// heavy / light pairing.
+template <bool DUAL, bool PLAIN = false>
 __device__ __forceinline__ Unit decode_item(const FwdParams& p, int u, int item) {
   Unit w;
   w.jbase = 0;
@@ -244,7 +250,7 @@ __device__ __forceinline__ Unit decode_item(const FwdParams& p, int u, int item)
   int qp;
   w.bh = u / p.units_per_head;
   const int b = u % p.units_per_head;
-  if (p.causal) {
+  if (p.causal && !PLAIN) {
     qp = item == 0 ? p.num_q_pairs - 1 - b : b;
   } else {
     qp = b;
@@ -271,6 +277,56 @@ __device__ __forceinline__ Unit decode_item(const FwdParams& p, int u, int item)
   return w;
 }
 
+// Split-mode step counts.  Query tile i sees min(nk, i + 1) key tiles under
+// the top-left causal mask (its last row is min(128 i + 127, Nq - 1)), so
+// pair qp needs min(nk, 2 qp + 2) steps, or min(nk, 2 qp + 1) when its second
+// tile lies past Nq; without the mask every pair needs nk.
+__device__ __forceinline__ int split_unit_steps(const FwdParams& p, int qp) {
+  if (!p.causal) return p.num_kv_tiles;
+  const int last_tile = (2 * qp + 1 < p.num_q_tiles) ? 2 * qp + 1 : 2 * qp;
+  return min(p.num_kv_tiles, last_tile + 1);
+}
+// Steps of the pairs before qp in a head (qp <= num_q_pairs - 1, so only
+// whole pairs): sum of min(nk, 2 q + 2) over q < qp = m (m + 1) + (qp - m) nk
+// with m = min(qp, nk / 2), the pairs whose count is not capped at nk.
+__device__ __forceinline__ long long split_head_prefix(const FwdParams& p, int qp) {
+  const long long nk = p.num_kv_tiles;
+  if (!p.causal) return static_cast<long long>(qp) * nk;
+  const long long m = min(static_cast<long long>(qp), nk / 2);
+  return m * (m + 1) + (qp - m) * nk;
+}
+// The pair whose steps contain step `rem` of a head (the inverse of the prefix).
+__device__ __forceinline__ int split_locate_pair(const FwdParams& p, long long rem) {
+  const long long nk = p.num_kv_tiles;
+  long long qp;
+  if (!p.causal) {
+    qp = rem / nk;
+  } else {
+    const long long a = nk / 2;
+    if (rem < a * (a + 1)) {
+      // largest m with m (m + 1) <= rem, then corrected for rounding
+      long long m = static_cast<long long>((sqrt(4.0 * static_cast<double>(rem) + 1.0) - 1.0) * 0.5);
+      while (m > 0 && m * (m + 1) > rem) --m;
+      while ((m + 1) * (m + 2) <= rem) ++m;
+      qp = m;
+    } else {
+      qp = a + (rem - a * (a + 1)) / nk;
+    }
+  }
+  return static_cast<int>(min(qp, static_cast<long long>(p.num_q_pairs - 1)));
+}
+// First flattened step of split unit u (= bh * num_q_pairs + qp).
+__device__ __forceinline__ long long split_unit_start(const FwdParams& p, int u) {
+  const int bh = u / p.num_q_pairs;
+  return static_cast<long long>(bh) * p.steps_per_head +
+         split_head_prefix(p, u - bh * p.num_q_pairs);
+}
+__device__ __forceinline__ int split_locate_unit(const FwdParams& p, long long step) {
+  const long long bh = step / p.steps_per_head;
+  return static_cast<int>(bh) * p.num_q_pairs +
+         split_locate_pair(p, step - bh * p.steps_per_head);
+}
+
 // Iterates the items of this CTA, identically in every role.
 template <bool SPLIT, bool DUAL>
 struct WorkCursor {
@@ -286,17 +342,16 @@ struct WorkCursor {
       // the 64-bit divisions run once per CTA, not once per item
       const long long begin = p.total_steps * blockIdx.x / gridDim.x;
       const long long end = p.total_steps * (blockIdx.x + 1) / gridDim.x;
-      const int nk = p.num_kv_tiles;
       item = items = 0;
       if (begin >= end) {
         u = 0;
         u_last = -1;
         return;
       }
-      u = static_cast<int>(begin / nk);
-      j_first = static_cast<int>(begin - static_cast<long long>(u) * nk);
-      u_last = static_cast<int>((end - 1) / nk);
-      j_end = static_cast<int>(end - static_cast<long long>(u_last) * nk);
+      u = split_locate_unit(p, begin);
+      j_first = static_cast<int>(begin - split_unit_start(p, u));
+      u_last = split_locate_unit(p, end - 1);
+      j_end = static_cast<int>(end - split_unit_start(p, u_last));
       pieces_of(p, u, j_first, piece_first, pieces_first, c_first_first);
       pieces_of(p, u_last, 0, piece_last, pieces_last, c_first_last);
     } else {
@@ -315,24 +370,26 @@ struct WorkCursor {
   // number of pieces, and the CTA holding piece 0.
   __device__ __forceinline__ static void pieces_of(const FwdParams& p, int uu, int j0, int& piece,
                                                    int& pieces, int& c_first) {
-    const int nk = p.num_kv_tiles;
-    const long long a = static_cast<long long>(uu) * nk;
+    const int steps = split_unit_steps(p, uu % p.num_q_pairs);
+    const long long a = split_unit_start(p, uu);
     const long long ca = starts_le(p, a);
     piece = static_cast<int>(starts_le(p, a + j0) - ca);
-    pieces = static_cast<int>(1 + starts_le(p, a + nk - 1) - ca);
+    pieces = static_cast<int>(1 + starts_le(p, a + steps - 1) - ca);
     c_first = static_cast<int>(ca);
   }
   __device__ __forceinline__ bool next(const FwdParams& p, Unit& w) {
     if constexpr (SPLIT) {
       if (u > u_last) return false;
-      const int nk = p.num_kv_tiles;
       const bool first = (item == 0);
       const int j0 = first ? j_first : 0;
-      const int j1 = (u == u_last) ? j_end : nk;
-      w = decode_item<false>(p, u, 0);
+      const int j1 = (u == u_last) ? j_end : split_unit_steps(p, u % p.num_q_pairs);
+      w = decode_item<false, true>(p, u, 0);
       w.jbase = j0;
-      w.n[0] = w.n[0] > 0 ? j1 - j0 : 0;
-      w.n[1] = w.n[1] > 0 ? j1 - j0 : 0;
+      // key tiles [j0, j1) of the unit; a query tile sees only those below
+      // its own count (under the causal mask the first tile of a pair sees
+      // one fewer than the second, and may see none of a late piece)
+      w.n[0] = max(0, min(j1, w.n[0]) - j0);
+      w.n[1] = max(0, min(j1, w.n[1]) - j0);
       w.nmax = max(w.n[0], w.n[1]);
       if (first) {
         w.piece = piece_first;
@@ -1098,7 +1155,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
         // --------------------------------------------------------- epilogue
         const bool in_range = row < p.Nq;
-        float lse_self = 0.f, inv_self = 0.f;  // this piece's statistics, for the merge
+        // this piece's statistics, for the merge; a piece in which this query
+        // tile sees no key (under the causal mask) has lse = -inf, weight 0
+        float lse_self = -INFINITY, inv_self = 0.f;
         if (n > 0) {
           if constexpr (NSB > 2) {
             ok = wait_count(smem_addr(smem + L::PV_DONE_OFF) + 4 * t, pv_handed, abort_flag,
@@ -1155,6 +1214,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             if (in_range) __stcg(p.ws_lse + wr, lse_row);
           }
           tc_fence_before();
+        } else if (SPLIT && w.pieces > 1) {
+          if (in_range) __stcg(p.ws_lse + ws_row(blockIdx.x, w.piece == 0 ? 1 : 0, t, r), -INFINITY);
         }
         if (SPLIT && w.pieces > 1) {
           // Both warpgroups publish their rows, then one thread counts the
@@ -1212,13 +1273,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                 float v[64];
                 if (k == w.piece) {
                   wk = w_self;
-                  uint32_t o[32];
 #pragma unroll
-                  for (int c0 = 0; c0 < 64; c0 += 32) {
-                    tmem_ld32(tO + 64 * h + c0, o);
-                    tmem_wait_ld_regs(o);
+                  for (int c = 0; c < 64; ++c) v[c] = 0.f;
+                  if (n > 0) {  // warp-uniform: the tile's own O is in TMEM
+                    uint32_t o[32];
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) v[c0 + c] = __uint_as_float(o[c]) * inv_self;
+                    for (int c0 = 0; c0 < 64; c0 += 32) {
+                      tmem_ld32(tO + 64 * h + c0, o);
+                      tmem_wait_ld_regs(o);
+#pragma unroll
+                      for (int c = 0; c < 32; ++c) v[c0 + c] = __uint_as_float(o[c]) * inv_self;
+                    }
                   }
                 } else {
                   const int slot = k == 0 ? 1 : 0;
@@ -1228,10 +1293,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                   if (in_range) {
                     wk = ex2_approx((__ldcg(p.ws_lse + ws_row(w.c_first + k, slot, t, r)) - lse_max) *
                                     1.4426950408889634f);
-                    const float* src = p.ws_o + ws_o_base(w.c_first + k, slot, t, D) +
-                                       static_cast<size_t>(64 * h) * BLOCK_M + r;
+                    if (wk != 0.f) {  // a piece that saw no key of this row wrote no O
+                      const float* src = p.ws_o + ws_o_base(w.c_first + k, slot, t, D) +
+                                         static_cast<size_t>(64 * h) * BLOCK_M + r;
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) v[c] = __ldcg(src + static_cast<size_t>(c) * BLOCK_M);
+                      for (int c = 0; c < 64; ++c) v[c] = __ldcg(src + static_cast<size_t>(c) * BLOCK_M);
+                    }
                   }
                 }
                 hsum += wk;

@@ -78,9 +78,11 @@ typedef struct {
   int stages;        /* K/V shared-memory ring slots                                      */
   long long qk_tile_products; /* 128x128 score tiles computed (incl. masked tail tiles)   */
   int split;         /* 1 if attn_fwd_ws would use split mode for these sizes (see below)  */
-  int split_grid;    /* CTAs launched in split mode: min(SM count, split_units * num_kv_tiles) */
+  int split_grid;    /* CTAs launched in split mode: min(SM count, split_steps)             */
   int split_units;   /* units split mode shares out: B * H * num_q_pairs (no dual units)  */
   long long workspace_bytes; /* workspace attn_fwd_ws needs for split mode; 0 if unused    */
+  long long split_steps;     /* key-tile steps split mode shares out: sum over the split units
+                                of the key tiles each query pair sees                       */
 } attn_plan_t;
 
 /*
@@ -111,11 +113,13 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
 /*
  * attn_fwd_ws -- attn_fwd with a caller-provided device workspace that enables split mode.
  *
- * For non-causal problems whose work units would fill the GPU unevenly (a ragged last wave,
- * or fewer units than SMs) and where the serial key-tile steps this saves outweigh the cost
- * of merging pieces (few units with many key tiles each, e.g. B = H = 1, N = 2000; attn_plan
- * reports the decision), the kernel divides the flattened (unit, key tile) range evenly over
- * the CTAs.  A unit cut by a range boundary
+ * For problems whose work units would fill the GPU unevenly (a ragged last wave, or fewer
+ * units than SMs) and where the serial key-tile steps this saves outweigh the cost of merging
+ * pieces (few units with many key tiles each, e.g. B = H = 1, N = 2000, causal or not;
+ * attn_plan reports the decision), the kernel divides the flattened (unit, key tile) range
+ * evenly over the CTAs.  A unit is one query pair of one (batch, head) with the key tiles
+ * its queries see (under the causal mask a pair's later tile sees i + 1 key tiles for
+ * query tile i, its first tile one fewer).  A unit cut by a range boundary
  * is computed in pieces; each piece writes its normalised O and its logsumexp to the
  * workspace and the last piece to finish merges them exactly with the log-domain identity
  * lse = ln sum_k exp(lse_k), O = sum_k exp(lse_k - lse) O_k (the saved-statistics

@@ -334,6 +334,28 @@ def test_split_many_pieces(B, H, Nq, Nk, d, dtype):
     assert _err(lse.double().numpy(), l_ref) <= LSE_TOL
 
 
+@pytest.mark.parametrize("B,H,Nq,Nk,d,dtype", [
+    (1, 1, 768, 768, 64, "fp16"),      # 2 causal units -> 12 key-tile steps on 12 CTAs
+    (1, 1, 2000, 2000, 64, "bf16"),    # 72 steps: first tiles of late pieces see no key
+    (1, 2, 4096, 4096, 128, "fp16"),   # d = 128, 544 steps on 148 CTAs
+    (2, 4, 1024, 1024, 64, "fp16"),
+    (1, 1, 3000, 1000, 64, "bf16"),    # Nq > Nk: later pairs see every key tile
+    (1, 2, 1000, 4000, 64, "bf16"),    # Nq < Nk: most key tiles hidden from every query
+])
+def test_split_causal(B, H, Nq, Nk, d, dtype):
+    assert A.attn_plan(B, H, Nq, Nk, d, 1, torch.cuda.get_device_properties(0).multi_processor_count)["split"] == 1
+    q, k, v = make_qkv(B, H, Nq, Nk, d, dtype, seed=Nq + 3 * Nk + d)
+    scale = 1.0 / math.sqrt(d)
+    o, lse, ws = _run_ws(q, k, v, True, scale)
+    assert ws is not None
+    o_ref, l_ref = oracle.attention_f64(q, k, v, scale, True)
+    assert _err(o.double().numpy(), o_ref) <= TOL[dtype]
+    assert _err(lse.double().numpy(), l_ref) <= LSE_TOL
+    # a second call on the same workspace gives the same bits (the counters were reset)
+    o2, lse2, _ = _run_ws(q, k, v, True, scale)
+    assert torch.equal(o, o2) and torch.equal(lse, lse2)
+
+
 def test_split_workspace_reuse_is_deterministic():
     """Reusing one workspace gives the same bits: each call leaves the counters at zero."""
     q, k, v = (t.cuda() for t in make_qkv(1, 2, 1500, 1500, 64, "fp16", seed=31))

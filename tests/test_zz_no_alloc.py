@@ -63,14 +63,22 @@ def test_noalloc_matches_workspace_entry(B, H, Nq, Nk, d, dtype):
         assert eo <= TOL[dtype] and el <= LSE_TOL, (eo, el)
 
 
-def test_noalloc_causal_needs_no_scratch():
-    q, k, v = (t.cuda() for t in make_qkv(1, 2, 700, 700, 64, "fp16", seed=3))
-    o_ref, l_ref = A.forward(q, k, v, causal=True)
-    for _ in range(2):
+@pytest.mark.parametrize("B,H,N,split", [(1, 2, 700, True), (16, 4, 700, False)])
+def test_noalloc_causal(B, H, N, split):
+    """Causal shapes: a small grid takes split mode from the fixed scratch and gives the bits of
+    attn_fwd_ws; a full grid needs no scratch and gives the bits of attn_fwd."""
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert A.attn_plan(B, H, N, N, 64, 1, sms)["split"] == int(split)
+    q, k, v = (t.cuda() for t in make_qkv(B, H, N, N, 64, "fp16", seed=3))
+    ws = A.workspace_for(q, k, True)
+    assert (ws is not None) == split
+    o_ref, l_ref = A.forward(q, k, v, causal=True, workspace=ws)
+    for _ in range(2):  # two calls in a row share (and must clear) the fixed scratch
         o = torch.empty_like(q)
-        lse = torch.empty((1, 2, 700), dtype=torch.float32, device="cuda")
+        lse = torch.empty((B, H, N), dtype=torch.float32, device="cuda")
         assert _call_noalloc(q, k, v, o, lse, True, 0.125, A.ATTN_FP16) == 0
         torch.cuda.synchronize()
+        assert A.attn_get_device_status()[0] == 0
         assert torch.equal(o, o_ref) and torch.equal(lse, l_ref)
 
 
