@@ -335,12 +335,12 @@ def test_split_many_pieces(B, H, Nq, Nk, d, dtype):
 
 
 @pytest.mark.parametrize("B,H,Nq,Nk,d,dtype", [
-    (1, 1, 768, 768, 64, "fp16"),      # 2 causal units -> 12 key-tile steps on 12 CTAs
+    (1, 1, 4096, 4096, 64, "fp16"),    # 8 causal units -> 272 key-tile steps on 148 CTAs
     (1, 1, 2000, 2000, 64, "bf16"),    # 72 steps: first tiles of late pieces see no key
     (1, 2, 4096, 4096, 128, "fp16"),   # d = 128, 544 steps on 148 CTAs
-    (2, 4, 1024, 1024, 64, "fp16"),
+    (1, 4, 2048, 2048, 64, "fp16"),
     (1, 1, 3000, 1000, 64, "bf16"),    # Nq > Nk: later pairs see every key tile
-    (1, 2, 1000, 4000, 64, "bf16"),    # Nq < Nk: most key tiles hidden from every query
+    (1, 1, 2500, 8000, 64, "bf16"),    # Nq < Nk: most key tiles hidden from every query
 ])
 def test_split_causal(B, H, Nq, Nk, d, dtype):
     assert A.attn_plan(B, H, Nq, Nk, d, 1, torch.cuda.get_device_properties(0).multi_processor_count)["split"] == 1

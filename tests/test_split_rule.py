@@ -4,7 +4,8 @@ A consistency check of a restated host formula (it calls no kernel): split
 mode is chosen when unit mode leaves the grid ragged (fewer units than SMs,
 or a last wave under 90 % full) and the serial key-tile steps it saves per
 CTA exceed its cost of merging pieces: about 3.5 + 0.56 steps per piece at
-d = 64 and 2.5 + 1.03 at d = 128.  Unit mode counts dual units (odd
+d = 64 and 2.5 + 1.03 at d = 128, 1.3 times that under the causal mask.
+Unit mode counts dual units (odd
 query-tile count, two or more heads, non-causal) and, under the causal mask,
 units of a heavy query pair plus its light mirror; split mode shares out
 plain units (one query pair of one head), each with the key tiles its later
@@ -49,7 +50,7 @@ def rule(B, H, Nq, Nk, d, causal, sms):
         return False
     grid_s = min(steps, sms)
     pieces = -(-max(per_pair) * grid_s // steps)
-    cost = 3.5 + 0.56 * pieces if d == 64 else 2.5 + 1.03 * pieces
+    cost = (3.5 + 0.56 * pieces if d == 64 else 2.5 + 1.03 * pieces) * (1.3 if causal else 1.0)
     return waves * unit_steps - (-(-steps // grid_s)) > cost
 
 

@@ -63,7 +63,7 @@ def test_noalloc_matches_workspace_entry(B, H, Nq, Nk, d, dtype):
         assert eo <= TOL[dtype] and el <= LSE_TOL, (eo, el)
 
 
-@pytest.mark.parametrize("B,H,N,split", [(1, 2, 700, True), (16, 4, 700, False)])
+@pytest.mark.parametrize("B,H,N,split", [(1, 2, 2000, True), (16, 4, 700, False)])
 def test_noalloc_causal(B, H, N, split):
     """Causal shapes: a small grid takes split mode from the fixed scratch and gives the bits of
     attn_fwd_ws; a full grid needs no scratch and gives the bits of attn_fwd."""
