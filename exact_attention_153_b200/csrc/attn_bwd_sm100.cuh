@@ -69,7 +69,12 @@ struct BwdSmem {
   static constexpr int STAGES = 2;
   static constexpr int DS_OFF = RING_OFF + STAGES * 2 * TILE_BYTES;  // dS^T, 2 slabs of 64 queries
   static constexpr int DS_BYTES = 2 * HALF_BYTES;
-  static constexpr int BAR_OFF = DS_OFF + DS_BYTES;
+  // At d = 64 each stage also holds the tile's 128 lse (base 2) and D values,
+  // copied in with Q_i and dO_i; d = 128 has no room and reads them from
+  // global memory.
+  static constexpr bool STATS_IN_SMEM = (D == 64);
+  static constexpr int STATS_OFF = DS_OFF + DS_BYTES;  // + stage * 1024: lse2[128], then D[128]
+  static constexpr int BAR_OFF = STATS_OFF + (STATS_IN_SMEM ? STAGES * 1024 : 0);
   // mbarriers
   static constexpr int KV_FULL = 0;
   static constexpr int RING_FULL = 1;                // + stage
@@ -275,7 +280,14 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (leader) {
         const int q0 = (i0 + n) * 128;
         const uint32_t dst = sbase + L::RING_OFF + s * 2 * L::TILE_BYTES;
-        mbar_arrive_expect_tx(bar(L::RING_FULL + s), 2 * L::TILE_BYTES);
+        mbar_arrive_expect_tx(bar(L::RING_FULL + s),
+                              2 * L::TILE_BYTES + (L::STATS_IN_SMEM ? 1024 : 0));
+        if constexpr (L::STATS_IN_SMEM) {
+          const size_t row0 = static_cast<size_t>(bh) * p.nq_pad + q0;  // 512-byte aligned
+          bulk_load(sbase + L::STATS_OFF + s * 1024, p.lse2 + row0, 512, bar(L::RING_FULL + s));
+          bulk_load(sbase + L::STATS_OFF + s * 1024 + 512, p.dsum + row0, 512,
+                    bar(L::RING_FULL + s));
+        }
 #pragma unroll
         for (int h = 0; h < D / 64; ++h) {
           tma_load_3d(dst + h * L::HALF_BYTES, &tm_q, bar(L::RING_FULL + s), h * 64, q0, bh);
@@ -438,10 +450,21 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     uint8_t* ds_tile = smem + L::DS_OFF;
     const float* lse2_bh = p.lse2 + static_cast<size_t>(bh) * p.nq_pad;
     const float* dsum_bh = p.dsum + static_cast<size_t>(bh) * p.nq_pad;
+    const float* stats_smem = reinterpret_cast<const float*>(smem + L::STATS_OFF);
     bool ok = true;
     for (int n = 0; ok && n < n_tiles; ++n) {
       const int q0 = (i0 + n) * 128;
       const int qw = q0 + 64 * w;  // first query of this warpgroup's columns
+      // d = 128: lane l holds the lse2 and D of queries qw + l and qw + 32 + l
+      // (coalesced loads issued before the wait); column c is then taken from
+      // lane c % 32 by a shuffle
+      float lse_lo = 0.f, lse_hi = 0.f, ds_lo = 0.f, ds_hi = 0.f;
+      if constexpr (!L::STATS_IN_SMEM) {
+        lse_lo = lse2_bh[qw + lane];
+        lse_hi = lse2_bh[qw + 32 + lane];
+        ds_lo = dsum_bh[qw + lane];
+        ds_hi = dsum_bh[qw + 32 + lane];
+      }
       ok = __all_sync(0xffffffffu, wait_phase(bar(L::S_READY), n & 1, abort_flag,
                                               SITE_SOFTMAX_S_FULL));
       if (!ok) break;
@@ -459,12 +482,33 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       // P = 2^(s * scale * log2 e - lse2); 0 for keys past Nk, queries past
       // Nq (lse2 = +inf there) and, causal, queries before the key
       uint32_t pk[32];
-      const float4* l4 = reinterpret_cast<const float4*>(lse2_bh + qw);
+      // the stage's lse2 / D landed with Q_i; these threads observe that
+      // stage's completed phase themselves before reading them (the stage is
+      // refilled only after this tile's dS is handed over, so the phase is
+      // unambiguous and already complete: S^T(n) was computed from it)
+      if constexpr (L::STATS_IN_SMEM) {
+        ok = __all_sync(0xffffffffu, wait_phase(bar(L::RING_FULL + n % L::STAGES),
+                                                (n / L::STAGES) & 1, abort_flag,
+                                                SITE_SOFTMAX_S_FULL));
+        if (!ok) break;
+      }
+      const float* stage_stats = stats_smem + (n % L::STAGES) * 256;
+      const float4* l4 = reinterpret_cast<const float4*>(stage_stats + 64 * w);
       const bool diag = p.causal && qw < key;  // some of these queries precede the key
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 lv = l4[c4];
-        const float lsv[4] = {lv.x, lv.y, lv.z, lv.w};
+        float lsv[4];
+        if constexpr (L::STATS_IN_SMEM) {
+          const float4 lv = l4[c4];
+          lsv[0] = lv.x;
+          lsv[1] = lv.y;
+          lsv[2] = lv.z;
+          lsv[3] = lv.w;
+        } else {
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            lsv[e] = __shfl_sync(0xffffffffu, c4 < 8 ? lse_lo : lse_hi, (4 * c4 + e) & 31);
+        }
         float pv[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
@@ -491,7 +535,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         if (!ok) break;
       }
       tc_fence_after();
-      const float4* d4 = reinterpret_cast<const float4*>(dsum_bh + qw);
+      const float4* d4 = reinterpret_cast<const float4*>(stage_stats + 128 + 64 * w);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t dp[32];
@@ -500,8 +544,18 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         uint32_t ds[16];
 #pragma unroll
         for (int c4 = 0; c4 < 8; ++c4) {
-          const float4 dv = d4[8 * half + c4];
-          const float dsv[4] = {dv.x, dv.y, dv.z, dv.w};
+          float dsv[4];
+          if constexpr (L::STATS_IN_SMEM) {
+            const float4 dv = d4[8 * half + c4];
+            dsv[0] = dv.x;
+            dsv[1] = dv.y;
+            dsv[2] = dv.z;
+            dsv[3] = dv.w;
+          } else {
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              dsv[e] = __shfl_sync(0xffffffffu, half ? ds_hi : ds_lo, (4 * c4 + e) & 31);
+          }
           float o[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {

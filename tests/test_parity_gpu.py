@@ -94,11 +94,15 @@ def test_many_units_persistent_loop():
 
 @pytest.mark.parametrize("idx", [0, 1])
 def test_workload_full_compare(idx):
+    import time
     w = WORKLOADS[idx]
     q, k, v = make_workload_qkv(w)
+    t0 = time.perf_counter()
     eo, el = _check_full(q, k, v, w.causal, w.scale, w.dtype)
+    dt = time.perf_counter() - t0
     print(f"\nPARITY {w.name}: max|dO| {eo:.3e} (tol {TOL[w.dtype]}), "
-          f"max|dlse| {el:.3e} (tol {LSE_TOL}), {w.B * w.H} (batch, head) slices")
+          f"max|dlse| {el:.3e} (tol {LSE_TOL}), {w.B * w.H} (batch, head) slices, "
+          f"oracle and GPU {dt:.1f} s in one process")
 
 
 @pytest.mark.parametrize("idx", [2, 3, 4])
@@ -110,13 +114,18 @@ def test_workload_full_parity(idx):
     every other case.
     """
     from tests.oracle_pool import compare_all_slices
+    import time
+    from tests.oracle_pool import workers
     w = WORKLOADS[idx]
     q, k, v = make_workload_qkv(w)
     o, lse = _run(q, k, v, w.causal, w.scale)
+    t0 = time.perf_counter()
     worst_o, worst_l, per_slice = compare_all_slices(q, k, v, o, lse, w.scale, w.causal)
+    dt = time.perf_counter() - t0
     assert len(per_slice) == w.B * w.H
     print(f"\nPARITY {w.name}: max|dO| {worst_o:.3e} (tol {TOL[w.dtype]}), "
-          f"max|dlse| {worst_l:.3e} (tol {LSE_TOL}), {len(per_slice)} (batch, head) slices")
+          f"max|dlse| {worst_l:.3e} (tol {LSE_TOL}), {len(per_slice)} (batch, head) slices, "
+          f"oracle {dt:.1f} s on {workers()} processes")
     assert worst_o <= TOL[w.dtype], f"O err {worst_o:.3e}"
     assert worst_l <= LSE_TOL, f"lse err {worst_l:.3e}"
 
