@@ -652,7 +652,8 @@ thread_local BwdMapCache t_do_map;
 std::atomic<bool> g_bwd_attr[kMaxDevices][2][2];  // [dev][d == 128][bf16]
 
 template <int D, bool BF16>
-int bwd_launch(const MapCache& maps, const CUtensorMap& m_do, const void* o, const void* dout,
+int bwd_launch(const MapCache& maps, const CUtensorMap& m_do, const CUtensorMap& m_dq,
+               const void* o, const void* dout,
                const float* lse, void* dq, const attn_sm100::BwdParams& prm, int dev, int sms,
                cudaStream_t stream) {
   using L = attn_sm100::BwdSmem<D>;
@@ -678,7 +679,7 @@ int bwd_launch(const MapCache& maps, const CUtensorMap& m_do, const void* o, con
       const_cast<float*>(prm.lse2), const_cast<float*>(prm.dsum), prm.dq_acc, prm.Nq, prm.nq_pad, BH);
   const long long grid = static_cast<long long>(prm.nk_tiles) * BH;
   main_kernel<<<static_cast<unsigned int>(grid), attn_sm100::BWD_THREADS, L::BYTES, stream>>>(
-      maps.mq, maps.mk, maps.mv, m_do, prm);
+      maps.mq, maps.mk, maps.mv, m_do, m_dq, prm);
   const long long n4 = BH * prm.Nq * (D / 4);
   const long long dq_blocks_needed = (n4 + 255) / 256;
   const int dq_blocks = static_cast<int>(dq_blocks_needed < 16LL * sms ? dq_blocks_needed : 16LL * sms);
@@ -746,13 +747,30 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
   prm.scale = scale;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // d = 64: the fp32 dQ accumulator as the 3-D map (64, Nq, B H) with 32-column
+  // x 128-row boxes and the 128-byte swizzle, the target of the bulk reductions
+  CUtensorMap m_dq;
+  if (d == 64) {
+    EncodeTiledFn enc = encode_fn();
+    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(Nq), static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {64 * 4, static_cast<cuuint64_t>(Nq) * 64 * 4};
+    const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(BLOCK_M), 1};
+    const cuuint32_t es[3] = {1, 1, 1};
+    if (enc == nullptr ||
+        enc(&m_dq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, prm.dq_acc, dims, strides, box, es,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return ATTN_ERR_CUDA;
+  } else {
+    m_dq = dm.m;  // unused at d = 128 (vector atomics)
+  }
   if (d == 64)
     return dtype == ATTN_BF16
-               ? bwd_launch<64, true>(*maps, dm.m, o, dout, lse, dq, prm, dev, info->sms, s)
-               : bwd_launch<64, false>(*maps, dm.m, o, dout, lse, dq, prm, dev, info->sms, s);
+               ? bwd_launch<64, true>(*maps, dm.m, m_dq, o, dout, lse, dq, prm, dev, info->sms, s)
+               : bwd_launch<64, false>(*maps, dm.m, m_dq, o, dout, lse, dq, prm, dev, info->sms, s);
   return dtype == ATTN_BF16
-             ? bwd_launch<128, true>(*maps, dm.m, o, dout, lse, dq, prm, dev, info->sms, s)
-             : bwd_launch<128, false>(*maps, dm.m, o, dout, lse, dq, prm, dev, info->sms, s);
+             ? bwd_launch<128, true>(*maps, dm.m, m_dq, o, dout, lse, dq, prm, dev, info->sms, s)
+             : bwd_launch<128, false>(*maps, dm.m, m_dq, o, dout, lse, dq, prm, dev, info->sms, s);
 }
 
 // ---------------------------------------------------------------------------

@@ -74,7 +74,13 @@ struct BwdSmem {
   // global memory.
   static constexpr bool STATS_IN_SMEM = (D == 64);
   static constexpr int STATS_OFF = DS_OFF + DS_BYTES;  // + stage * 1024: lse2[128], then D[128]
-  static constexpr int BAR_OFF = STATS_OFF + (STATS_IN_SMEM ? STAGES * 1024 : 0);
+  // At d = 64 the readout stages dQ_ij (128 rows x 64 fp32, two 32-column
+  // halves with the 128-byte swizzle) in one of two 32 KB slots and adds it
+  // to the accumulator with two TMA bulk reductions; d = 128 has no room and
+  // adds with per-thread vector atomics.
+  static constexpr bool DQ_BULK = (D == 64);
+  static constexpr int DQ_OFF = STATS_OFF + (STATS_IN_SMEM ? STAGES * 1024 : 0);  // + slot * 32 KB
+  static constexpr int BAR_OFF = DQ_OFF + (DQ_BULK ? 2 * 32768 : 0);
   // mbarriers
   static constexpr int KV_FULL = 0;
   static constexpr int RING_FULL = 1;                // + stage
@@ -87,7 +93,8 @@ struct BwdSmem {
   static constexpr int DQ_FREE = DQ_READY + 1;    // 128 readout threads arrive
   static constexpr int DONE = DQ_FREE + 1;        // every MMA done
   static constexpr int SYNC = DONE + 1;           // rendezvous of the 256 softmax threads
-  static constexpr int NUM_BARS = SYNC + 1;
+  static constexpr int RO_SYNC = SYNC + 1;        // rendezvous of the 128 readout threads
+  static constexpr int NUM_BARS = RO_SYNC + 1;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // TMEM address, abort flag
   static constexpr int BYTES = MISC_OFF + 16 + 1024;      // + slack to align the base to 1 KB
   static_assert(BYTES <= 232448, "shared memory budget");
@@ -205,7 +212,7 @@ template <int D, bool BF16>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using L = BwdSmem<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -238,6 +245,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     mbar_init(bar(L::DQ_FREE), 128);
     mbar_init(bar(L::DONE), 1);
     mbar_init(bar(L::SYNC), 256);
+    mbar_init(bar(L::RO_SYNC), 128);
     *abort_flag = 0;
     fence_mbarrier_init();
   }
@@ -409,32 +417,70 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     // ------------------------------------------------------------- dQ readout
     const int r = (warp - 8) * 32 + lane;  // query row within the tile
     const uint32_t t_dq = tmem_base + L::DP_COL + (static_cast<uint32_t>((warp - 8) * 32) << 16);
+    const bool issuer = (threadIdx.x == 8 * 32);  // issues and waits for the bulk reductions
+    uint32_t ro_phase = 0;
+    auto ro_sync = [&]() -> bool {  // bounded rendezvous of the 128 readout threads
+      mbar_arrive(bar(L::RO_SYNC));
+      const bool ok = wait_phase(bar(L::RO_SYNC), ro_phase, abort_flag, SITE_SOFTMAX_SYNC);
+      ro_phase ^= 1;
+      return __all_sync(0xffffffffu, ok);
+    };
     for (int n = 0; n < n_tiles; ++n) {
       const bool ok = __all_sync(0xffffffffu, wait_phase(bar(L::DQ_READY), n & 1, abort_flag,
                                                          SITE_SOFTMAX_O_READY));
       if (!ok) break;
       tc_fence_after();
-      const int q = (i0 + n) * 128 + r;
-      float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.Nq + q) * D;
-      // 64 columns at a time; the columns are handed back after the last load
-#pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 64) {
+      const int q0 = (i0 + n) * 128;
+      const int q = q0 + r;
+      if constexpr (L::DQ_BULK) {
         uint32_t v[64];
-        tmem_ld32(t_dq + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
-        tmem_ld32(t_dq + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+        tmem_ld32(t_dq, *reinterpret_cast<uint32_t(*)[32]>(v));
+        tmem_ld32(t_dq + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
         tmem_wait_ld_regs(v);
-        if (c0 + 64 == D) {
-          tc_fence_before();
-          mbar_arrive(bar(L::DQ_FREE));
-        }
-        if (q < p.Nq) {
+        tc_fence_before();
+        mbar_arrive(bar(L::DQ_FREE));
+        // slot n & 1 was last read by the reductions of tile n - 2
+        if (issuer && n >= 2) bulk_wait_group_read<1>();
+        if (!ro_sync()) break;
+        uint8_t* slot = smem + L::DQ_OFF + (n & 1) * 32768;
 #pragma unroll
-          for (int c = 0; c < 64; c += 4)
-            red_add_v4(dst + c0 + c, __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                       __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch)
+            *reinterpret_cast<uint4*>(slot + h * 16384 + r * 128 + ((ch ^ (r & 7)) << 4)) =
+                make_uint4(v[32 * h + 4 * ch], v[32 * h + 4 * ch + 1], v[32 * h + 4 * ch + 2],
+                           v[32 * h + 4 * ch + 3]);
+        fence_proxy_async_shared();
+        if (!ro_sync()) break;
+        if (issuer) {
+          // rows past Nq fall outside the tensor and are not written
+          tma_reduce_add_3d(&tm_dq, sbase + L::DQ_OFF + (n & 1) * 32768, 0, q0, bh);
+          tma_reduce_add_3d(&tm_dq, sbase + L::DQ_OFF + (n & 1) * 32768 + 16384, 32, q0, bh);
+          bulk_commit_group();
+        }
+      } else {
+        float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.Nq + q) * D;
+        // 64 columns at a time; the columns are handed back after the last load
+#pragma unroll
+        for (int c0 = 0; c0 < D; c0 += 64) {
+          uint32_t v[64];
+          tmem_ld32(t_dq + c0, *reinterpret_cast<uint32_t(*)[32]>(v));
+          tmem_ld32(t_dq + c0 + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
+          tmem_wait_ld_regs(v);
+          if (c0 + 64 == D) {
+            tc_fence_before();
+            mbar_arrive(bar(L::DQ_FREE));
+          }
+          if (q < p.Nq) {
+#pragma unroll
+            for (int c = 0; c < 64; c += 4)
+              red_add_v4(dst + c0 + c, __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                         __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+          }
         }
       }
     }
+    if (L::DQ_BULK && issuer) bulk_wait_group<0>();  // every reduction done before the CTA exits
   } else {
     // ------------------------------------------------------------- softmax
     // Thread = key row r of the tile; warpgroup w takes query columns
