@@ -747,13 +747,15 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
   prm.scale = scale;
   prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // d = 64: the fp32 dQ accumulator as the 3-D map (64, Nq, B H) with 32-column
-  // x 128-row boxes and the 128-byte swizzle, the target of the bulk reductions
+  // the fp32 dQ accumulator as the 3-D map (d, Nq, B H) with 32-column x
+  // 128-row boxes and the 128-byte swizzle, the target of the bulk reductions
   CUtensorMap m_dq;
-  if (d == 64) {
+  {
     EncodeTiledFn enc = encode_fn();
-    const cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(Nq), static_cast<cuuint64_t>(BH)};
-    const cuuint64_t strides[2] = {64 * 4, static_cast<cuuint64_t>(Nq) * 64 * 4};
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(Nq),
+                                static_cast<cuuint64_t>(BH)};
+    const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4,
+                                   static_cast<cuuint64_t>(Nq) * d * 4};
     const cuuint32_t box[3] = {32, static_cast<cuuint32_t>(BLOCK_M), 1};
     const cuuint32_t es[3] = {1, 1, 1};
     if (enc == nullptr ||
@@ -761,8 +763,6 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return ATTN_ERR_CUDA;
-  } else {
-    m_dq = dm.m;  // unused at d = 128 (vector atomics)
   }
   if (d == 64)
     return dtype == ATTN_BF16

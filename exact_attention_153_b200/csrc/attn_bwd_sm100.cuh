@@ -74,13 +74,16 @@ struct BwdSmem {
   // global memory.
   static constexpr bool STATS_IN_SMEM = (D == 64);
   static constexpr int STATS_OFF = DS_OFF + DS_BYTES;  // + stage * 1024: lse2[128], then D[128]
-  // At d = 64 the readout stages dQ_ij (128 rows x 64 fp32, two 32-column
-  // halves with the 128-byte swizzle) in one of two 32 KB slots and adds it
-  // to the accumulator with two TMA bulk reductions; d = 128 has no room and
-  // adds with per-thread vector atomics.
-  static constexpr bool DQ_BULK = (D == 64);
+  // The readout adds each dQ_ij tile (128 rows x D fp32, 32-column boxes with
+  // the 128-byte swizzle) to the accumulator with TMA bulk reductions from
+  // shared memory.  At d = 64 it stages the tile in one of two 32 KB slots of
+  // its own; at d = 128, which has no room for them, in the ring stage of the
+  // tile itself (Q_i and dO_i take exactly 64 KB, and every MMA that read them
+  // is done when dQ_ij is), and the readout, not the MMA warp, then hands the
+  // stage back to the loader once the reductions have read it.
+  static constexpr bool DQ_IN_STAGE = (D == 128);
   static constexpr int DQ_OFF = STATS_OFF + (STATS_IN_SMEM ? STAGES * 1024 : 0);  // + slot * 32 KB
-  static constexpr int BAR_OFF = DQ_OFF + (DQ_BULK ? 2 * 32768 : 0);
+  static constexpr int BAR_OFF = DQ_OFF + (DQ_IN_STAGE ? 0 : 2 * 32768);
   // mbarriers
   static constexpr int KV_FULL = 0;
   static constexpr int RING_FULL = 1;                // + stage
@@ -405,7 +408,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           mma_ss(t_dp, ds_mn + kk * (2048 >> 4), k_mn + kk * (2048 >> 4), IDESC_QA,
                  kk > 0 ? 1u : 0u);
         mma_commit(bar(L::DQ_READY));
-        mma_commit(bar(L::RING_EMPTY + s));
+        if (!L::DQ_IN_STAGE) mma_commit(bar(L::RING_EMPTY + s));  // else the readout frees it
       }
       __syncwarp();
     }
@@ -432,7 +435,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tc_fence_after();
       const int q0 = (i0 + n) * 128;
       const int q = q0 + r;
-      if constexpr (L::DQ_BULK) {
+      if constexpr (!L::DQ_IN_STAGE) {
         uint32_t v[64];
         tmem_ld32(t_dq, *reinterpret_cast<uint32_t(*)[32]>(v));
         tmem_ld32(t_dq + 32, *reinterpret_cast<uint32_t(*)[32]>(v + 32));
@@ -459,8 +462,10 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           bulk_commit_group();
         }
       } else {
-        float* dst = p.dq_acc + (static_cast<size_t>(bh) * p.Nq + q) * D;
-        // 64 columns at a time; the columns are handed back after the last load
+        // stage the tile in the ring stage of tile n (free: DQ_READY(n) follows
+        // every MMA of tile n), four 32-column boxes of 16 KB
+        const int s = n % L::STAGES;
+        uint8_t* stage = smem + L::RING_OFF + s * 2 * L::TILE_BYTES;
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 64) {
           uint32_t v[64];
@@ -471,16 +476,28 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             tc_fence_before();
             mbar_arrive(bar(L::DQ_FREE));
           }
-          if (q < p.Nq) {
 #pragma unroll
-            for (int c = 0; c < 64; c += 4)
-              red_add_v4(dst + c0 + c, __uint_as_float(v[c]), __uint_as_float(v[c + 1]),
-                         __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
-          }
+          for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+              *reinterpret_cast<uint4*>(stage + (c0 / 32 + h) * 16384 + r * 128 +
+                                        ((ch ^ (r & 7)) << 4)) =
+                  make_uint4(v[32 * h + 4 * ch], v[32 * h + 4 * ch + 1], v[32 * h + 4 * ch + 2],
+                             v[32 * h + 4 * ch + 3]);
+        }
+        fence_proxy_async_shared();
+        if (!ro_sync()) break;
+        if (issuer) {
+          const uint32_t src = sbase + L::RING_OFF + s * 2 * L::TILE_BYTES;
+#pragma unroll
+          for (int b = 0; b < D / 32; ++b) tma_reduce_add_3d(&tm_dq, src + b * 16384, 32 * b, q0, bh);
+          bulk_commit_group();
+          bulk_wait_group_read<0>();  // the stage has been read: the loader may refill it
+          mbar_arrive(bar(L::RING_EMPTY + s));
         }
       }
     }
-    if (L::DQ_BULK && issuer) bulk_wait_group<0>();  // every reduction done before the CTA exits
+    if (issuer) bulk_wait_group<0>();  // every reduction done before the CTA exits
   } else {
     // ------------------------------------------------------------- softmax
     // Thread = key row r of the tile; warpgroup w takes query columns

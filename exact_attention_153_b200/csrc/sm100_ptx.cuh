@@ -310,7 +310,7 @@ __device__ __forceinline__ void regs_decrease() {
 }
 
 // ---------------------------------------------------------------------------
-// Proxy fence, vector reduction
+// Proxy fence
 // ---------------------------------------------------------------------------
 // Makes this thread's generic-proxy shared-memory writes visible to the async
 // proxy (tcgen05.mma operands read from shared memory).
@@ -318,12 +318,6 @@ __device__ __forceinline__ void fence_proxy_async_shared() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
-// *p += {a, b, c, d} as one relaxed atomic reduction (16-byte aligned p).
-__device__ __forceinline__ void red_add_v4(float* p, float a, float b, float c, float d) {
-  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
-               "f"(d)
-               : "memory");
-}
 
 // ---------------------------------------------------------------------------
 // MUFU and conversions (single PTX instructions)
