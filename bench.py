@@ -273,6 +273,8 @@ def main():
                     help="skip the context timings of the other workloads")
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of float64 oracle work for cpu_baseline")
+    ap.add_argument("--part", choices=["forward", "backward", "block"], default="forward",
+                    help="with --kernel-only: which path to run (for ncu captures)")
     ap.add_argument("--kernel-only", action="store_true",
                     help="time only the device loop (no e2e, CPU baseline or context timings);"
                          " used for ncu captures")
@@ -283,6 +285,8 @@ def main():
     w = workload(args.workload)
     if args.impl == "reference":
         return run_reference(args, w)
+    if args.kernel_only and args.part != "forward":
+        return run_part(args, w)
 
     import torch
     import torch.distributed as dist
@@ -575,6 +579,43 @@ def graph_per_call_us(attn, torch, w, q, k, v, o, lse, ws, calls: int, replays: 
         times.append(e0.elapsed_time(e1) * 1e3 / calls)
     del g
     return statistics.median(times)
+
+
+def run_part(args, w):
+    """--kernel-only for the backward or the block: W warm-up and K timed calls on one GPU."""
+    import torch
+    import exact_attention_153_b200 as attn
+    from seeded_inputs import make_block_inputs, make_grad_out, make_workload_qkv
+    dev = torch.device("cuda", 0)
+    if args.part == "backward":
+        q, k, v = (t.to(dev) for t in make_workload_qkv(w))
+        do = make_grad_out(w.B, w.H, w.Nq, w.d, w.dtype, w.seed).to(dev)
+        o, lse = attn.forward(q, k, v, causal=w.causal)
+        ws = torch.empty(attn.attn_bwd_workspace_size(w.B, w.H, w.Nq, w.Nk, w.d),
+                         dtype=torch.uint8, device=dev)
+        grads = (torch.empty_like(q), torch.empty_like(k), torch.empty_like(v))
+        fn = lambda: attn.backward(q, k, v, o, lse, do, causal=w.causal, workspace=ws, out=grads)
+        flops = backward_flops(w)
+    else:
+        C = w.H * w.d
+        x, w_qkv, b_qkv, w_o, b_o = (t.to(dev) if t is not None else None
+                                     for t in make_block_inputs(w.B, w.Nq, w.H, w.d, C, w.dtype, 7))
+        fn = lambda: attn.block_forward(x, w_qkv, b_qkv, w_o, b_o, w.H, causal=w.causal)
+        flops = 8.0 * w.B * w.Nq * C * C + w.flops
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / args.steps
+    print(json.dumps({"workload": w.name, "part": args.part, "us_per_call": round(ms * 1e3, 2),
+                      "tflops": round(flops / (ms * 1e-3) / 1e12, 2), "steps": args.steps}),
+          flush=True)
+    return 0
 
 
 def context_timings(attn, torch, dev, peaks, steps=50, warmup=5, device_index=0):

@@ -227,10 +227,19 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::MISC_OFF + 4);
   auto bar = [&](int i) -> uint32_t { return sbase + L::BAR_OFF + 8u * i; };
 
-  // key tile j of (batch, head) bh; all heads' tile 0 first (the heaviest
-  // tiles under the causal mask start first)
-  const int j = static_cast<int>(blockIdx.x / p.BH);
-  const int bh = static_cast<int>(blockIdx.x - static_cast<long long>(j) * p.BH);
+  // key tile j of (batch, head) bh.  Without the mask all heads' tile 0 come
+  // first, so CTAs that run together add their dQ tiles into different heads;
+  // under the causal mask a head's key tiles are adjacent, so the CTAs that
+  // read its Q and dO run together and share them through L2 (measured: -2 %
+  // and -8 % on the causal workloads, +3 % on the non-causal ones)
+  int j, bh;
+  if (p.causal) {
+    bh = static_cast<int>(blockIdx.x / p.nk_tiles);
+    j = static_cast<int>(blockIdx.x - static_cast<long long>(bh) * p.nk_tiles);
+  } else {
+    j = static_cast<int>(blockIdx.x / p.BH);
+    bh = static_cast<int>(blockIdx.x - static_cast<long long>(j) * p.BH);
+  }
   const int i0 = bwd_first_q_tile(p, j);
   const int n_tiles = p.nq_tiles > i0 ? p.nq_tiles - i0 : 0;
 
