@@ -13,3 +13,4 @@ from .backward import (  # noqa: F401
     row_dot,
 )
 from .block import attention_block_f64, linear, merge_heads, split_qkv  # noqa: F401
+from .fp8 import attention_fp8_f64, decode_e4m3, dequantize_e4m3, untranspose_v  # noqa: F401

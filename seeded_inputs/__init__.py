@@ -31,7 +31,7 @@ from dataclasses import dataclass, field
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "workload", "make_qkv", "dtype_of", "make_grad_out",
-           "make_workload_qkv", "make_block_inputs"]
+           "make_workload_qkv", "make_block_inputs", "make_fp8_qkv"]
 
 _DTYPES = {"fp16": torch.float16, "bf16": torch.bfloat16}
 
@@ -156,3 +156,35 @@ def make_block_inputs(B: int, N: int, H: int, d: int, C_out: int, dtype: str, se
     b_o = 0.1 * torch.randn((C_out,), generator=g, dtype=torch.float32)
     b_qkv = 0.1 * torch.randn((3 * C,), generator=g, dtype=torch.float32) if qkv_bias else None
     return x, w_qkv, b_qkv, w_o, b_o
+
+
+def make_fp8_qkv(B: int, H: int, Nq: int, Nk: int, d: int, seed: int, qk_scale: float = 1.0):
+    """Seeded e4m3 inputs with one scale factor per tensor.
+
+    Q, K, V are drawn as in ``make_qkv`` (float32, Q and K times
+    ``qk_scale``); each tensor x is stored as the e4m3 codes of
+    x * (448 / max|x|) (torch's round-to-nearest-even cast, so the largest
+    magnitude lands on 448, the format's largest finite value) with descale
+    max|x| / 448, which turns codes back into values.  V is stored
+    transposed, [B, H, d, Nk].  Returns CPU tensors
+    (q8 [B,H,Nq,d], k8 [B,H,Nk,d], vt8 [B,H,d,Nk]) of torch.float8_e4m3fn
+    and the descales (q_descale, k_descale, v_descale) as Python floats.
+    """
+    g = torch.Generator(device="cpu")
+    g.manual_seed(int(seed))
+    q = torch.randn((B, H, Nq, d), generator=g, dtype=torch.float32)
+    k = torch.randn((B, H, Nk, d), generator=g, dtype=torch.float32)
+    v = torch.randn((B, H, Nk, d), generator=g, dtype=torch.float32)
+    if qk_scale != 1.0:
+        q.mul_(qk_scale)
+        k.mul_(qk_scale)
+
+    def quantize(x):
+        amax = float(x.abs().max())
+        amax = amax if amax > 0 else 1.0
+        return (x * (448.0 / amax)).to(torch.float8_e4m3fn).contiguous(), amax / 448.0
+
+    q8, qs = quantize(q)
+    k8, ks = quantize(k)
+    vt8, vs = quantize(v.transpose(-1, -2).contiguous())
+    return q8, k8, vt8, (qs, ks, vs)
