@@ -273,7 +273,7 @@ def main():
                     help="skip the context timings of the other workloads")
     ap.add_argument("--cpu-budget", type=float, default=12.0,
                     help="seconds of float64 oracle work for cpu_baseline")
-    ap.add_argument("--part", choices=["forward", "backward", "block"], default="forward",
+    ap.add_argument("--part", choices=["forward", "backward", "block", "fp8"], default="forward",
                     help="with --kernel-only: which path to run (for ncu captures)")
     ap.add_argument("--kernel-only", action="store_true",
                     help="time only the device loop (no e2e, CPU baseline or context timings);"
@@ -400,12 +400,14 @@ def main():
     per_workload = None
     backward = None
     blocks = None
+    fp8 = None
     cpu = None
     if rank == 0 and world == 1 and not args.no_per_workload:
         per_workload = context_timings(attn, torch, dev, peaks, steps=args.steps,
                                        warmup=args.warmup, device_index=local)
         backward = backward_timings(attn, torch, dev, peaks, warmup=args.warmup)
         blocks = block_timings(attn, torch, dev, peaks, warmup=args.warmup)
+        fp8 = fp8_timings(attn, torch, dev, peaks, warmup=args.warmup)
     if rank == 0:
         flops, dt, done = time_oracle_sample(w, q, k, v, budget_s=args.cpu_budget)
         cpu = {"value": flops / dt / 1e12, "unit": "TFLOPS", "cores": blas_threads() or cpu_cores(),
@@ -440,6 +442,8 @@ def main():
             line["backward"] = backward
         if blocks is not None:
             line["block"] = blocks
+        if fp8 is not None:
+            line["fp8"] = fp8
         print(json.dumps(line), flush=True)
     if world > 1:
         dist.destroy_process_group()
@@ -485,6 +489,72 @@ def backward_timings(attn, torch, dev, peaks, steps=20, warmup=3):
                        "frac": round(tf / peaks["bf16_tflops"], 4), "bound": "tensor",
                        "launches": 3}
         del q, k, v, do, o, lse, ws, grads
+        torch.cuda.empty_cache()
+    return out
+
+
+FP8_CONFIGS = [
+    # name, B, H, N, causal, qk_scale: the d = 128 workload, and the 80x80 map's 256
+    # channels as two heads of d = 128
+    ("long_context_32k", 1, 32, 32768, True, 0.5),
+    ("yolo_highres_80x80_b16_d128", 16, 2, 6400, False, 1.0),
+]
+
+
+def fp8_config(name):
+    for c in FP8_CONFIGS:
+        if c[0] == name:
+            return c
+    raise KeyError(name)
+
+
+def fp8_timings(attn, torch, dev, peaks, steps=20, warmup=3):
+    """µs/call (L2 flushed before each call; median, p10, p90) of the e4m3 forward, next to
+    the bf16 forward on inputs of the same shape.  Its roofline peak is the measured bf16
+    GEMM rate times 2, the nominal e4m3 / bf16 tensor-rate ratio (4.5 / 2.25 PFLOP/s)."""
+    from seeded_inputs import make_fp8_qkv, make_qkv
+    out = {}
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    peak = 2.0 * peaks["bf16_tflops"]
+
+    def timed(fn):
+        for _ in range(max(3, warmup)):
+            fn()
+        torch.cuda.synchronize()
+        times = []
+        for _ in range(steps):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            fn()
+            e1.record()
+            torch.cuda.synchronize()
+            times.append(e0.elapsed_time(e1) * 1e3)
+        return percentiles(times)
+
+    for name, B, H, N, causal, qk in FP8_CONFIGS:
+        q8, k8, vt8, ds = make_fp8_qkv(B, H, N, N, 128, seed=1005, qk_scale=qk)
+        q8, k8, vt8 = q8.to(dev), k8.to(dev), vt8.to(dev)
+        ws = attn.workspace_for(q8, k8, causal)
+        o = torch.empty((B, H, N, 128), dtype=torch.bfloat16, device=dev)
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+        st8 = timed(lambda: attn.forward_fp8(q8, k8, vt8, ds, causal=causal, out=o, lse=lse,
+                                             workspace=ws))
+        del q8, k8, vt8
+        q, k, v = (t.to(dev) for t in make_qkv(B, H, N, N, 128, "bf16", seed=1005, qk_scale=qk))
+        ws16 = attn.workspace_for(q, k, causal)
+        st16 = timed(lambda: attn.forward(q, k, v, causal=causal, out=o, lse=lse,
+                                          workspace=ws16))
+        flops = 4.0 * B * H * N * N * 128 * (0.5 if causal else 1.0)
+        tf = flops / (st8["median"] * 1e-6) / 1e12
+        out[name] = {"B": B, "H": H, "N": N, "d": 128, "causal": causal,
+                     "us_per_call": round(st8["median"], 2), "us_p10": round(st8["p10"], 2),
+                     "us_p90": round(st8["p90"], 2), "tflops": round(tf, 2),
+                     "frac": round(tf / peak, 4), "peak": round(peak, 1),
+                     "peak_source": "measured bf16 x 2 (nominal e4m3 / bf16 ratio)",
+                     "bf16_us_per_call": round(st16["median"], 2),
+                     "speedup_vs_bf16": round(st16["median"] / st8["median"], 3)}
+        del q, k, v, o, lse, ws, ws16
         torch.cuda.empty_cache()
     return out
 
@@ -587,7 +657,15 @@ def run_part(args, w):
     import exact_attention_153_b200 as attn
     from seeded_inputs import make_block_inputs, make_grad_out, make_workload_qkv
     dev = torch.device("cuda", 0)
-    if args.part == "backward":
+    if args.part == "fp8":
+        from seeded_inputs import make_fp8_qkv
+        _, B, H, N, causal, qk = fp8_config(w.name if w.d == 128 else "yolo_highres_80x80_b16_d128")
+        q8, k8, vt8, ds = (x.to(dev) if hasattr(x, "to") else x
+                           for x in make_fp8_qkv(B, H, N, N, 128, seed=1005, qk_scale=qk))
+        ws = attn.workspace_for(q8, k8, causal)
+        fn = lambda: attn.forward_fp8(q8, k8, vt8, ds, causal=causal, workspace=ws)
+        flops = 4.0 * B * H * N * N * 128 * (0.5 if causal else 1.0)
+    elif args.part == "backward":
         q, k, v = (t.to(dev) for t in make_workload_qkv(w))
         do = make_grad_out(w.B, w.H, w.Nq, w.d, w.dtype, w.seed).to(dev)
         o, lse = attn.forward(q, k, v, causal=w.causal)

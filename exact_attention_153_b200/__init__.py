@@ -24,6 +24,7 @@ __all__ = [
     "forward_host", "STATUS_NAMES", "attn_fwd_ws", "attn_workspace_size", "workspace_for",
     "attn_fwd_noalloc", "attn_bwd", "attn_bwd_workspace_size", "backward",
     "attn_qkv_proj", "attn_out_proj", "attn_block_fwd", "qkv_proj", "out_proj", "block_forward",
+    "attn_fwd_fp8", "forward_fp8",
 ]
 
 ATTN_FP16 = 0
@@ -80,6 +81,9 @@ def lib() -> ctypes.CDLL:
         L.attn_fwd_ws.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp, ctypes.c_size_t,
                                   vp]
         L.attn_fwd_ws.restype = i
+        L.attn_fwd_fp8.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, f, f, f, i, vp,
+                                   ctypes.c_size_t, vp]
+        L.attn_fwd_fp8.restype = i
         L.attn_workspace_size.argtypes = [i, i, i, i, i, i, ctypes.POINTER(ctypes.c_size_t)]
         L.attn_workspace_size.restype = i
         L.attn_fwd_noalloc.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, i, i, vp]
@@ -123,6 +127,14 @@ def attn_fwd_ws(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, workspac
     """Raw ``attn_fwd_ws``: attn_fwd with a device workspace (split mode)."""
     return lib().attn_fwd_ws(q, k, v, o, lse, B, H, Nq, Nk, d, float(scale), int(causal), dtype,
                              workspace, ws_bytes, stream)
+
+
+def attn_fwd_fp8(q, k, vt, o, lse, B, H, Nq, Nk, d, scale, q_descale, k_descale, v_descale,
+                 causal, workspace, ws_bytes, stream) -> int:
+    """Raw ``attn_fwd_fp8``: e4m3 q, k and transposed v with per-tensor descales, bf16 o."""
+    return lib().attn_fwd_fp8(q, k, vt, o, lse, B, H, Nq, Nk, d, float(scale), float(q_descale),
+                              float(k_descale), float(v_descale), int(causal), workspace,
+                              ws_bytes, stream)
 
 
 def attn_fwd_noalloc(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, stream) -> int:
@@ -275,6 +287,48 @@ def forward(q, k, v, causal: bool = False, scale: float | None = None, out=None,
                          workspace.numel() * workspace.element_size(), _stream_handle(stream))
     if st != 0:
         raise AttnError(st)
+    return out, lse
+
+
+def forward_fp8(q8, k8, vt8, descales, causal: bool = False, scale: float | None = None,
+                out=None, lse=None, return_lse: bool = True, stream=None, workspace=None):
+    """FP8 attention forward: e4m3 q8 [B, H, Nq, 128], k8 [B, H, Nk, 128] and V transposed,
+    vt8 [B, H, 128, Nk] (Nk a multiple of 16), with ``descales`` = (q, k, v) factors that turn
+    codes into values.  Returns (o bf16 [B, H, Nq, 128], lse fp32 [B, H, Nq]).
+
+    The FP8 path of FlashAttention-3 ("一个反直觉的事实", ai2ai.xin, section
+    "FlashAttention-3的进一步增强", item 2).
+    """
+    import torch
+    if q8.dim() != 4 or k8.dim() != 4 or vt8.dim() != 4:
+        raise ValueError("q8, k8 must be [B, H, N, d] and vt8 [B, H, d, Nk]")
+    B, H, Nq, d = q8.shape
+    Nk = k8.shape[2]
+    if k8.shape != (B, H, Nk, d) or vt8.shape != (B, H, d, Nk):
+        raise ValueError(f"shape mismatch: q8 {tuple(q8.shape)} k8 {tuple(k8.shape)} "
+                         f"vt8 {tuple(vt8.shape)}")
+    if not (q8.is_cuda and k8.is_cuda and vt8.is_cuda):
+        raise ValueError("q8, k8, vt8 must be CUDA tensors (no CPU path exists)")
+    for name, t in (("q8", q8), ("k8", k8), ("vt8", vt8)):
+        if t.dtype != torch.float8_e4m3fn:
+            raise TypeError(f"{name} must be torch.float8_e4m3fn")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty((B, H, Nq, d), dtype=torch.bfloat16, device=q8.device)
+    if lse is None and return_lse:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q8.device)
+    qs, ks, vs = descales
+    st = attn_fwd_fp8(q8.data_ptr(), k8.data_ptr(), vt8.data_ptr(), out.data_ptr(),
+                      lse.data_ptr() if lse is not None else None, B, H, Nq, Nk, d, scale,
+                      qs, ks, vs, causal,
+                      workspace.data_ptr() if workspace is not None else None,
+                      workspace.numel() * workspace.element_size() if workspace is not None else 0,
+                      _stream_handle(stream))
+    if st != 0:
+        raise AttnError(st, "attn_fwd_fp8")
     return out, lse
 
 

@@ -53,8 +53,9 @@ struct DeviceInfo {
   bool probed = false;
   bool supported = false;
   int sms = 0;
-  // [d==128][bf16][unit, dual-unit, split kernel]: the shared-memory attribute is set
-  std::atomic<bool> smem_attr[2][2][3] = {};
+  // [d = 64, d = 128, d = 128 e4m3][bf16][unit, dual-unit, split kernel]: the
+  // shared-memory attribute is set
+  std::atomic<bool> smem_attr[3][2][3] = {};
 };
 
 std::mutex g_dev_mutex;
@@ -214,25 +215,37 @@ int current_device(int* dev_out, DeviceInfo** info_out) {
   return ATTN_OK;
 }
 
-// 3-D view (d, N, B*H) of a [B, H, N, d] tensor; boxes of 64 columns x 128
-// rows with the 128-byte swizzle the tcgen05 descriptors expect.  Rows past
-// N read as zero, so ragged tails never touch the next head.
-bool encode_map(CUtensorMap* map, const void* ptr, int N, long long BH, int d, int dtype) {
+// Internal element-type code of e4m3 operands (attn_fwd_fp8): keeps their
+// cached tensor maps apart from 16-bit maps of the same buffers.
+constexpr int kDtypeE4M3 = 2;
+
+// 3-D view (cols, rows, B*H) of a [B, H, rows, cols] tensor; boxes of 128
+// bytes x 128 rows (64 fp16 / bf16 or 128 e4m3 columns) with the 128-byte
+// swizzle the tcgen05 descriptors expect.  Rows past `rows` and columns past
+// `cols` read as zero, so ragged tails never touch the next head.
+bool encode_rows(CUtensorMap* map, const void* ptr, long long rows, long long BH, int cols,
+                 int dtype) {
   EncodeTiledFn enc = encode_fn();
   if (enc == nullptr) return false;
-  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+  const cuuint64_t elem = dtype == kDtypeE4M3 ? 1 : 2;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
                               static_cast<cuuint64_t>(BH)};
-  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
-                                 static_cast<cuuint64_t>(N) * static_cast<cuuint64_t>(d) * 2};
-  const cuuint32_t box[3] = {64, static_cast<cuuint32_t>(BLOCK_M), 1};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * elem,
+                                 static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols) * elem};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(128 / elem), static_cast<cuuint32_t>(BLOCK_M), 1};
   const cuuint32_t elem_strides[3] = {1, 1, 1};
-  const CUresult r = enc(map,
-                         dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
-                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                         3, const_cast<void*>(ptr), dims, strides, box, elem_strides,
+  const CUtensorMapDataType type = dtype == kDtypeE4M3 ? CU_TENSOR_MAP_DATA_TYPE_UINT8
+                                   : dtype == ATTN_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                        : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const CUresult r = enc(map, type, 3, const_cast<void*>(ptr), dims, strides, box, elem_strides,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
+}
+
+// [B, H, N, d] Q, K or V
+bool encode_map(CUtensorMap* map, const void* ptr, int N, long long BH, int d, int dtype) {
+  return encode_rows(map, ptr, N, BH, d, dtype);
 }
 
 // Per-thread cache of recent calls' tensor maps: repeated calls on the same
@@ -265,20 +278,23 @@ const MapCache* cached_maps(const void* q, const void* k, const void* v, int Nq,
   MapCache& mc = set.e[set.next];
   set.next = (set.next + 1) % kMapCacheEntries;
   mc.q = nullptr;  // invalid until all three encodes succeed
+  // e4m3: v is Vt [B, H, d, Nk], read in tiles of 128 keys x d rows
   if (!encode_map(&mc.mq, q, Nq, BH, d, dtype) || !encode_map(&mc.mk, k, Nk, BH, d, dtype) ||
-      !encode_map(&mc.mv, v, Nk, BH, d, dtype))
+      !(dtype == kDtypeE4M3 ? encode_rows(&mc.mv, v, d, BH, Nk, dtype)
+                            : encode_map(&mc.mv, v, Nk, BH, d, dtype)))
     return nullptr;
   mc.q = q; mc.k = k; mc.v = v;
   mc.Nq = Nq; mc.Nk = Nk; mc.d = d; mc.dtype = dtype; mc.dev = dev; mc.BH = BH;
   return &mc;
 }
 
-template <int D, bool BF16, bool SPLIT, bool DUAL>
+template <int D, bool BF16, bool SPLIT, bool DUAL, bool FP8>
 int launch_one(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo& info,
                cudaStream_t stream) {
-  auto kernel = attn_sm100::attn_fwd_kernel<D, BF16, SPLIT, DUAL>;
-  constexpr int smem = SmemLayout<D>::BYTES;
-  std::atomic<bool>& attr = info.smem_attr[D == 128][BF16][SPLIT ? 2 : (DUAL ? 1 : 0)];
+  auto kernel = attn_sm100::attn_fwd_kernel<D, BF16, SPLIT, DUAL, FP8>;
+  constexpr int smem = SmemLayout<D, FP8>::BYTES;
+  std::atomic<bool>& attr =
+      info.smem_attr[FP8 ? 2 : (D == 128 ? 1 : 0)][BF16][SPLIT ? 2 : (DUAL ? 1 : 0)];
   if (!attr.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lock(g_dev_mutex);
     if (!attr.load(std::memory_order_relaxed)) {
@@ -296,18 +312,27 @@ int launch_one(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo&
 
 // Split mode and unit mode with dual units are separate instantiations, so
 // the plain unit-mode kernel carries none of their bookkeeping.
-template <int D, bool BF16>
+template <int D, bool BF16, bool FP8 = false>
 int launch(const MapCache& maps, const FwdParams& prm, int grid, DeviceInfo& info,
            cudaStream_t stream) {
-  if (prm.split) return launch_one<D, BF16, true, false>(maps, prm, grid, info, stream);
-  if (prm.dual_base >= 0) return launch_one<D, BF16, false, true>(maps, prm, grid, info, stream);
-  return launch_one<D, BF16, false, false>(maps, prm, grid, info, stream);
+  if (prm.split) return launch_one<D, BF16, true, false, FP8>(maps, prm, grid, info, stream);
+  if (prm.dual_base >= 0)
+    return launch_one<D, BF16, false, true, FP8>(maps, prm, grid, info, stream);
+  return launch_one<D, BF16, false, false, FP8>(maps, prm, grid, info, stream);
 }
 
+// The extra arguments of the e4m3 forward.
+struct Fp8Scales {
+  float q_descale, k_descale, v_descale;
+};
+
+// `f8` != nullptr: e4m3 operands (q, k and v = Vt), bf16 output; `dtype` is
+// then ATTN_BF16, the output type, and the caller has validated the e4m3
+// arguments.
 static int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, int B,
                     int H, int Nq, int Nk, int d, float scale, int causal, int dtype,
                     void* workspace, size_t workspace_bytes, attn_stream_t stream,
-                    int stall_site = 0) {
+                    int stall_site = 0, const Fp8Scales* f8 = nullptr) {
   int st = check_args(q, k, v, o, lse, B, H, Nq, Nk, d, scale, dtype);
   if (st != ATTN_OK) return st;
   int dev = -1;
@@ -319,7 +344,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   fill_plan(B, H, Nq, Nk, d, causal, info->sms, &plan);
   const long long BH = static_cast<long long>(B) * H;
 
-  const MapCache* maps = cached_maps(q, k, v, Nq, Nk, BH, d, dtype, dev);
+  const MapCache* maps = cached_maps(q, k, v, Nq, Nk, BH, d, f8 ? kDtypeE4M3 : dtype, dev);
   if (maps == nullptr) return ATTN_ERR_CUDA;
   const MapCache& mc = *maps;
 
@@ -336,7 +361,9 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
   prm.dual_base = plan.dual_units > 0 ? plan.num_units - plan.dual_units : -1;
   prm.last_q0 = (plan.num_q_tiles - 1) * BLOCK_M;
   prm.causal = causal ? 1 : 0;
-  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+  prm.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634 *
+                                      (f8 ? static_cast<double>(f8->q_descale) * f8->k_descale : 1.0));
+  prm.o_scale = f8 ? f8->v_descale : 1.f;
   prm.split = 0;
   prm.total_steps = 0;
   prm.num_q_tiles = plan.num_q_tiles;
@@ -366,6 +393,7 @@ static int fwd_impl(const void* q, const void* k, const void* v, void* o, float*
     // workspace) and every completed call leaves them at zero again
     prm.ws_count = reinterpret_cast<unsigned int*>(ws + rows * (d + 1) * sizeof(float));
   }
+  if (f8) return launch<128, true, true>(mc, prm, grid, *info, s);
   if (d == 64)
     return dtype == ATTN_BF16 ? launch<64, true>(mc, prm, grid, *info, s)
                               : launch<64, false>(mc, prm, grid, *info, s);
@@ -448,6 +476,23 @@ int attn_fwd_stall_test(const void* q, const void* k, const void* v, void* o, fl
   if (stall_site < 1 || stall_site > 4) return ATTN_ERR_SHAPE;
   return fwd_impl(q, k, v, o, lse, B, H, Nq, Nk, d, scale, causal, dtype, workspace,
                   workspace_bytes, stream, stall_site);
+}
+
+int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* lse, int B, int H,
+                 int Nq, int Nk, int d, float scale, float q_descale, float k_descale,
+                 float v_descale, int causal, void* workspace, size_t workspace_bytes,
+                 attn_stream_t stream) {
+  if (q == nullptr || k == nullptr || vt == nullptr || o == nullptr) return ATTN_ERR_NULL;
+  if (d != 128) return ATTN_ERR_HEAD_DIM;
+  if (B < 1 || H < 1 || Nq < 1 || Nk < 1 || Nk % 16 != 0) return ATTN_ERR_SHAPE;
+  for (float f : {q_descale, k_descale, v_descale})
+    if (!std::isfinite(f) || !(f > 0.f)) return ATTN_ERR_SCALE;
+  // the folded score scale must stay a finite, positive fp32 value
+  const double sl2 = static_cast<double>(scale) * q_descale * k_descale;
+  if (!std::isfinite(scale) || !(sl2 > 1e-30) || !(sl2 < 1e30)) return ATTN_ERR_SCALE;
+  const Fp8Scales f8{q_descale, k_descale, v_descale};
+  return fwd_impl(q, k, vt, o, lse, B, H, Nq, Nk, d, scale, causal, ATTN_BF16, workspace,
+                  workspace_bytes, stream, 0, &f8);
 }
 
 int attn_workspace_size(int B, int H, int Nq, int Nk, int d, int causal, size_t* bytes) {

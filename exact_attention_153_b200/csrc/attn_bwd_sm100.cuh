@@ -443,7 +443,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       if (!ok) break;
       tc_fence_after();
       const int q0 = (i0 + n) * 128;
-      const int q = q0 + r;
       if constexpr (!L::DQ_IN_STAGE) {
         uint32_t v[64];
         tmem_ld32(t_dq, *reinterpret_cast<uint32_t(*)[32]>(v));

@@ -82,9 +82,11 @@ constexpr float RESCALE_LOG2 = 8.0f;  // lazy-rescale threshold for the running 
 // Of every 16 key pairs in a 32-key chunk, this many take 2^x from a
 // polynomial on the FMA pipe and the rest from the MUFU ex2 unit, so the two
 // pipes share the exponentials.  At d = 64 the MUFU bounds the softmax; at
-// d = 128 the tensor core does, and the polynomial only costs issue slots.
-template <int D>
-__host__ __device__ constexpr int exp_poly_pairs() { return D == 64 ? 4 : 0; }
+// d = 128 the tensor core does, and the polynomial only costs issue slots --
+// except with e4m3 operands, whose MMAs take half the time, so the MUFU
+// bounds that softmax as well.
+template <int D, bool FP8 = false>
+__host__ __device__ constexpr int exp_poly_pairs() { return (D == 64 || FP8) ? 4 : 0; }
 
 // Device status word: 0 = healthy; otherwise 0x80000000 | site.
 __device__ unsigned int g_attn_status = 0;
@@ -125,7 +127,8 @@ struct FwdParams {
   int dual_base;
   int last_q0;
   int causal;
-  float scale_log2; // scale * log2(e)
+  float scale_log2; // scale * log2(e) (e4m3 operands: times the Q and K descales)
+  float o_scale;    // e4m3 operands: the V descale, applied with 1 / l; unused otherwise
   // Split mode.  Every unit is one query pair of one (batch, head); its key
   // tiles are flattened into total_steps = B H * steps_per_head steps (a
   // pair needs num_kv_tiles of them, or under the causal mask only the tiles
@@ -144,18 +147,24 @@ struct FwdParams {
   int stall_site;          // StallSite; 0 except through the test hook
 };
 
-template <int D>
+// FP8: e4m3 operands (d = 128 only).  A tile row is then 128 one-byte
+// elements, one 128-byte swizzle row, and V arrives transposed (Vt tiles of
+// d rows x 128 keys), so both MMAs read K-major operands.
+template <int D, bool FP8 = false>
 struct SmemLayout {
-  static constexpr int HALF_BYTES = BLOCK_M * 64 * 2;  // one 64-column, 128-byte-swizzled slab
-  static constexpr int HALVES = D / 64;
+  // one 128-row slab of 128-byte rows, 128-byte swizzled: 64 fp16 / bf16 or 128 e4m3 columns
+  static constexpr int HALF_BYTES = BLOCK_M * 128;
+  static constexpr int HALVES = FP8 ? 1 : D / 64;
+  static_assert(!FP8 || D == 128, "e4m3 tiles hold 128 one-byte columns");
   static constexpr int TILE_BYTES = HALVES * HALF_BYTES;
   // separate K and V rings, filled in the order the MMA warp consumes them
-  static constexpr int K_STAGES = (D == 64) ? 4 : 3;
-  static constexpr int V_STAGES = (D == 64) ? 4 : 2;
-  // Q: slots of two tiles.  Two slots at d = 64, so the next item's Q tiles
-  // load while the current item runs and its first S does not wait for them;
-  // one at d = 128, where shared memory has no room for a second.
-  static constexpr int Q_SLOTS = (D == 64) ? 2 : 1;
+  static constexpr int K_STAGES = (D == 64 || FP8) ? 4 : 3;
+  static constexpr int V_STAGES = (D == 64 || FP8) ? 4 : 2;
+  // Q: slots of two tiles.  Two slots at d = 64 and with e4m3 tiles, so the
+  // next item's Q tiles load while the current item runs and its first S
+  // does not wait for them; one at d = 128 (16-bit), where shared memory has
+  // no room for a second.
+  static constexpr int Q_SLOTS = (D == 64 || FP8) ? 2 : 1;
   static constexpr int Q_OFF = 0;
   static constexpr int K_OFF = Q_OFF + Q_SLOTS * 2 * TILE_BYTES;
   static constexpr int V_OFF = K_OFF + K_STAGES * TILE_BYTES;
@@ -558,11 +567,14 @@ __device__ __forceinline__ bool wait_phase(uint32_t bar, uint32_t parity, volati
 // DUAL: the unit-mode kernel for problems with dual units (an odd number of
 // query tiles per head); the other unit-mode problems run the DUAL = false
 // instantiation, which carries none of the dual-unit bookkeeping.
-template <int D, bool BF16, bool SPLIT, bool DUAL>
+// FP8: Q, K and Vt are e4m3 (tm_v then maps Vt [B H, d, Nk]); O is written as
+// bf16 (BF16 must be true).
+template <int D, bool BF16, bool SPLIT, bool DUAL, bool FP8 = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     attn_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using L = SmemLayout<D>;
+  static_assert(!FP8 || (D == 128 && BF16), "e4m3 operands: d = 128, bf16 output");
+  using L = SmemLayout<D, FP8>;
   constexpr int NSB = L::NSB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -690,10 +702,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             }
             if (leader) {
               mbar_arrive_expect_tx(bar(full0 + st), L::TILE_BYTES);
+              if (FP8 && !is_k) {  // Vt tile: all d rows, keys (jbase + j) * 128 ..
+                tma_load_3d(ring + st * L::TILE_BYTES, map, bar(full0 + st),
+                            (w.jbase + j) * BLOCK_N, 0, bh);
+              } else {
 #pragma unroll
-              for (int h = 0; h < L::HALVES; ++h)
-                tma_load_3d(ring + st * L::TILE_BYTES + h * L::HALF_BYTES, map, bar(full0 + st),
-                            h * 64, (w.jbase + j) * BLOCK_N, bh);
+                for (int h = 0; h < L::HALVES; ++h)
+                  tma_load_3d(ring + st * L::TILE_BYTES + h * L::HALF_BYTES, map, bar(full0 + st),
+                              h * 64, (w.jbase + j) * BLOCK_N, bh);
+              }
             }
             __syncwarp();
             ++pos;
@@ -719,8 +736,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // issues O_t += P(g) V_j as soon as the softmax has written P(g).  Each
       // warp only waits on its own inputs, so one waiting for the softmax
       // does not hold back the other's work.
-      constexpr uint32_t IDESC_S = idesc_f16(BF16, false, false, BLOCK_M, BLOCK_N);
-      constexpr uint32_t IDESC_O = idesc_f16(BF16, false, true, BLOCK_M, D);
+      constexpr uint32_t IDESC_S =
+          FP8 ? idesc_e4m3(BLOCK_M, BLOCK_N) : idesc_f16(BF16, false, false, BLOCK_M, BLOCK_N);
+      constexpr uint32_t IDESC_O = FP8 ? idesc_e4m3(BLOCK_M, D) : idesc_f16(BF16, false, true, BLOCK_M, D);
       // S: both operands K-major (head dim contiguous), 128-byte swizzle,
       // 8-row groups 1024 bytes apart; each k-step covers 16 elements = 32
       // bytes of a 128-byte row, the head dim > 64 continues in the next 16 KB
@@ -731,8 +749,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint64_t k_desc = sw128_desc(k_smem, 16, 1024);
       // P V: P from TMEM (16 keys = 8 columns per k-step), V MN-major (head
       // dim contiguous): 8-key groups 1024 bytes apart, 64-column slabs 16 KB
-      // apart; each k-step advances 16 keys = 2 KB.
-      const uint64_t v_desc = sw128_desc(v_smem, L::HALF_BYTES, 1024);
+      // apart; each k-step advances 16 keys = 2 KB.  e4m3: S and P V both take
+      // 32 elements = 32 bytes per k-step; P from TMEM (32 keys = 8 columns),
+      // Vt K-major like K (keys contiguous, d rows in 8-row groups 1 KB apart).
+      const uint64_t v_desc =
+          FP8 ? sw128_desc(v_smem, 16, 1024) : sw128_desc(v_smem, L::HALF_BYTES, 1024);
       const uint32_t tmem_s = tmem_base + L::S_COL;
       const uint32_t tmem_o = tmem_base + L::O_COL;
       // With only two S/P buffers (d = 128) the next S of a tile must reuse
@@ -787,10 +808,16 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const uint64_t a = q_item + static_cast<uint32_t>(sp.t * (L::TILE_BYTES >> 4));
               const uint64_t bd = k_desc + st * static_cast<uint32_t>(L::TILE_BYTES >> 4);
               if (leader) {
+                if constexpr (FP8) {
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                  const uint32_t off = ((kk / 4) * L::HALF_BYTES + (kk % 4) * 32) >> 4;
-                  mma_ss(tmem_s + 128 * b, a + off, bd + off, IDESC_S, kk > 0 ? 1u : 0u);
+                  for (int kk = 0; kk < D / 32; ++kk)
+                    mma_ss_f8(tmem_s + 128 * b, a + kk * 2, bd + kk * 2, IDESC_S, kk > 0 ? 1u : 0u);
+                } else {
+#pragma unroll
+                  for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t off = ((kk / 4) * L::HALF_BYTES + (kk % 4) * 32) >> 4;
+                    mma_ss(tmem_s + 128 * b, a + off, bd + off, IDESC_S, kk > 0 ? 1u : 0u);
+                  }
                 }
                 mma_commit(bar(L::S_FULL + 2 * b + sp.t));
                 if (last_use<DUAL>(w, sp)) mma_commit(bar(L::K_EMPTY + st));
@@ -819,10 +846,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               tc_fence_after();
               const uint64_t bd = v_desc + st * static_cast<uint32_t>(L::TILE_BYTES >> 4);
               if (leader) {
+                if constexpr (FP8) {
 #pragma unroll
-                for (int kk = 0; kk < BLOCK_N / 16; ++kk)
-                  mma_ts(tmem_o + D * sp.t, tmem_s + 128 * b + kk * 8, bd + kk * (2048 >> 4),
-                         IDESC_O, (sp.j > 0 || kk > 0) ? 1u : 0u);
+                  for (int kk = 0; kk < BLOCK_N / 32; ++kk)
+                    mma_ts_f8(tmem_o + D * sp.t, tmem_s + 128 * b + kk * 8, bd + kk * 2, IDESC_O,
+                              (sp.j > 0 || kk > 0) ? 1u : 0u);
+                } else {
+#pragma unroll
+                  for (int kk = 0; kk < BLOCK_N / 16; ++kk)
+                    mma_ts(tmem_o + D * sp.t, tmem_s + 128 * b + kk * 8, bd + kk * (2048 >> 4),
+                           IDESC_O, (sp.j > 0 || kk > 0) ? 1u : 0u);
+                }
                 // in-order issue: S_t(j + 1) completing already implies this
                 // P V completed, so only the tile's last P V is signalled
                 if (sp.j + 1 == (sp.t ? w.n[1] : w.n[0])) mma_commit(bar(L::O_READY + sp.t));
@@ -1094,10 +1128,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
             // P = 2^(s * scale * log2 e - m), packed two keys per 32-bit TMEM
             // column (even key in the low half), written over S in 16-column
-            // chunks so each chunk's S registers die as it is stored.
+            // chunks so each chunk's S registers die as it is stored.  e4m3:
+            // four keys per column (lowest key in the low byte), 8-column
+            // chunks; P < 2^RESCALE_LOG2 = 256 stays inside e4m3's range.
             float sum0 = 0.f, sum1 = 0.f;
 #pragma unroll
             for (int chunk = 0; chunk < 4; ++chunk) {
+              if constexpr (FP8) {
+                uint32_t pk[8];
+#pragma unroll
+                for (int c4 = 0; c4 < 8; ++c4) {
+                  float e[4];
+#pragma unroll
+                  for (int h = 0; h < 2; ++h) {
+                    const int c = 2 * c4 + h;  // key pair within the chunk
+                    float x0, x1;
+                    fma2(x0, x1, s[32 * chunk + 2 * c], s[32 * chunk + 2 * c + 1], sl2, sl2, neg_m,
+                         neg_m);
+                    if (c < exp_poly_pairs<D, FP8>()) {
+                      exp2_poly2(e[2 * h], e[2 * h + 1], x0, x1);
+                    } else {
+                      e[2 * h] = ex2_approx(x0);
+                      e[2 * h + 1] = ex2_approx(x1);
+                    }
+                    add2(sum0, sum1, sum0, sum1, e[2 * h], e[2 * h + 1]);
+                  }
+                  pk[c4] = pack4_e4m3(e[0], e[1], e[2], e[3]);
+                }
+                tmem_st8(tS + 8 * chunk, pk);
+                continue;
+              }
               uint32_t pk[16];
 #pragma unroll
               for (int c = 0; c < 16; ++c) {
@@ -1169,7 +1229,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           ok = __all_sync(0xffffffffu, ok);
           if (!ok) break;
           tc_fence_after();
-          const float inv_l = 1.f / l;
+          const float inv_l = (FP8 ? p.o_scale : 1.f) / l;
           const float lse_row = (m + lg2_approx(l)) * 0.69314718055994531f;
           lse_self = lse_row;
           inv_self = inv_l;

@@ -149,6 +149,37 @@ int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse
 int attn_workspace_size(int B, int H, int Nq, int Nk, int d, int causal, size_t* bytes);
 
 /*
+ * attn_fwd_fp8 -- attn_fwd_ws with 8-bit floating-point (e4m3) Q, K and V.
+ *
+ * "一个反直觉的事实：大模型推理的瓶颈不是计算，而是显存" (ai2ai.xin), section
+ * "FlashAttention-3的进一步增强", item 2: the attention runs on FP8 operands at half the
+ * memory of 16-bit ones.  Each input is an e4m3 tensor with one descale factor: the value
+ * an element stands for is e4m3(code) * descale.  The result is the exact attention of those
+ * values, O = softmax(scale * Q K^T) V with lse as in attn_fwd, computed with fp32
+ * accumulation and softmax statistics; P is rounded to e4m3 (relative error at most 2^-4,
+ * absolute at most 2^-10 relative to the running row maximum) before the P V product, and
+ * O is rounded once to bf16.
+ *
+ *   q   device, [B, H, Nq, d] e4m3 codes (one byte each), contiguous.
+ *   k   device, [B, H, Nk, d] e4m3 codes, contiguous.
+ *   vt  device, V TRANSPOSED: [B, H, d, Nk] e4m3 codes, contiguous (keys innermost, so
+ *       both products read their operands along the contracted axis).
+ *   o   device, [B, H, Nq, d] bf16 output.  lse as attn_fwd (nullable).
+ *   d   128 (the only head size of this entry point).  Nk a multiple of 16 (the byte
+ *       stride of a vt row must be a multiple of 16).
+ *   q_descale, k_descale, v_descale  finite and > 0; scale * q_descale * k_descale must be
+ *       a normal fp32 value.
+ *   workspace, workspace_bytes  as attn_fwd_ws (attn_workspace_size with d = 128).
+ * Errors, in this order: ATTN_ERR_NULL, ATTN_ERR_HEAD_DIM (d != 128), ATTN_ERR_SHAPE (also
+ * Nk % 16 != 0), ATTN_ERR_SCALE (descales), then the checks of attn_fwd (ATTN_ERR_ALIGN:
+ * q, k, vt, o 16-byte aligned).  On any error nothing is enqueued.  Asynchrony as attn_fwd.
+ */
+int attn_fwd_fp8(const void* q, const void* k, const void* vt, void* o, float* lse, int B, int H,
+                 int Nq, int Nk, int d, float scale, float q_descale, float k_descale,
+                 float v_descale, int causal, void* workspace, size_t workspace_bytes,
+                 attn_stream_t stream);
+
+/*
  * attn_fwd_noalloc -- attn_fwd_ws without a caller workspace and without any allocation.
  *
  * The pages have no counterpart to this entry point; it exists for callers that cannot

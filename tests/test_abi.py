@@ -36,7 +36,7 @@ def test_header_declares_the_boundary():
         "attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_noalloc", "attn_fwd_host",
         "attn_fwd_stall_test", "attn_plan", "attn_get_device_status", "attn_strerror",
         "attn_version", "attn_bwd", "attn_bwd_workspace_size", "attn_qkv_proj", "attn_out_proj",
-        "attn_block_fwd"])
+        "attn_block_fwd", "attn_fwd_fp8"])
 
 
 def test_every_declared_symbol_is_exported():
@@ -227,6 +227,36 @@ def test_bwd_workspace_size():
     assert A.attn_bwd_workspace_size(1, 1, 128, 1, 128) == 128 * 128 * 4 + 2 * 128 * 4
     with pytest.raises(A.AttnError):
         A.attn_bwd_workspace_size(1, 1, 128, 1, 80)
+
+
+# ------------------------------------------------------------------ e4m3 forward arguments
+
+FP8 = dict(q=0x10000, k=0x20000, vt=0x30000, o=0x40000, lse=None, B=1, H=2, Nq=300, Nk=512,
+           d=128, scale=0.088, qs=0.01, ks=0.02, vs=0.03, causal=0, ws=None, ws_bytes=0)
+
+
+def call_fp8(**kw):
+    a = dict(FP8)
+    a.update(kw)
+    return A.attn_fwd_fp8(a["q"], a["k"], a["vt"], a["o"], a["lse"], a["B"], a["H"], a["Nq"],
+                          a["Nk"], a["d"], a["scale"], a["qs"], a["ks"], a["vs"], a["causal"],
+                          a["ws"], a["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), 1), (dict(vt=None), 1), (dict(o=None), 1),
+    (dict(d=64), 3), (dict(d=256), 3),
+    (dict(Nq=0), 2), (dict(Nk=0), 2), (dict(Nk=500), 2), (dict(B=0), 2),
+    (dict(qs=0.0), 6), (dict(ks=-1.0), 6), (dict(vs=float("nan")), 6), (dict(qs=float("inf")), 6),
+    (dict(scale=0.0), 6), (dict(scale=1e-20, qs=1e-10, ks=1e-10), 6),
+    (dict(q=0x10008), 5), (dict(vt=0x30004), 5), (dict(o=0x40002), 5), (dict(lse=0x50002), 5),
+    (dict(), 8),  # valid arguments, no usable device here: ATTN_ERR_CUDA, never a CPU path
+])
+def test_fp8_argument_errors(kw, code):
+    import torch
+    if code == 8 and torch.cuda.is_available():
+        pytest.skip("a device is present")
+    assert call_fp8(**kw) == code
 
 
 # ------------------------------------------------------------------ projection arguments
