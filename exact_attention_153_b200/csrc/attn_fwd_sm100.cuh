@@ -474,13 +474,15 @@ __device__ __forceinline__ bool last_use(const Unit& w, SeqPos s) {
 }
 
 // P for one 128-key row: p = 2^(s * sl2 + neg_m), packed two keys per word
-// (even key low), and the fp32 sum of the unrounded values.  Of every 16 key
-// pairs, exp_poly_pairs<D>() take 2^x from the FMA-pipe polynomial.
-// d = 64 (bound by the softmax) tries the running max as it stands before
-// computing a row max; at d = 128 the extra registers of that path cost more
-// than it saves.
-template <int D>
-__host__ __device__ constexpr bool kStaleMaxFirst() { return D == 64; }
+// (even key low; e4m3: four keys per word, lowest key in the low byte), and
+// the fp32 sum of the unrounded values.  Of every 16 key pairs,
+// exp_poly_pairs<D, FP8>() take 2^x from the FMA-pipe polynomial.
+// d = 64 and e4m3 operands (both bound by the softmax) try the running max
+// as it stands before computing a row max; at d = 128 with 16-bit operands
+// the extra registers of that path cost more than it saves (e4m3 P needs
+// half the packed registers, 32 words per row).
+template <int D, bool FP8 = false>
+__host__ __device__ constexpr bool kStaleMaxFirst() { return D == 64 || FP8; }
 
 // With the running max as it stands (STALE) x has no upper bound.  The
 // MUFU's 2^x overflows to +inf for x >= 128, which the caller's sum check
@@ -492,16 +494,17 @@ __host__ __device__ constexpr bool kStaleMaxFirst() { return D == 64; }
 // check rejects).  Without STALE, x <= RESCALE_LOG2 by construction.
 constexpr float POLY_X_LIMIT = 64.0f;
 
-template <int D, bool BF16, bool STALE>
+template <int D, bool BF16, bool STALE, bool FP8 = false>
 __device__ __forceinline__ float exp_row(const float (&s)[128], float sl2, float neg_m,
-                                         uint32_t (&pk)[64], float& xp_max) {
+                                         uint32_t (&pk)[FP8 ? 32 : 64], float& xp_max) {
   float sum0 = 0.f, sum1 = 0.f;
   float xm = -INFINITY;
+  float prev0 = 0.f, prev1 = 0.f;
 #pragma unroll
   for (int i = 0; i < 64; ++i) {
     float x0, x1, a, bb;
     fma2(x0, x1, s[2 * i], s[2 * i + 1], sl2, sl2, neg_m, neg_m);
-    if (i % 16 < exp_poly_pairs<D>()) {
+    if (i % 16 < exp_poly_pairs<D, FP8>()) {
       if constexpr (STALE) xm = max3(xm, x0, x1);
       exp2_poly2(a, bb, x0, x1);  // FMA pipe, in parallel with the MUFU ones
     } else {
@@ -509,7 +512,16 @@ __device__ __forceinline__ float exp_row(const float (&s)[128], float sl2, float
       bb = ex2_approx(x1);
     }
     add2(sum0, sum1, sum0, sum1, a, bb);
-    pk[i] = pack2<BF16>(a, bb);
+    if constexpr (FP8) {
+      if (i % 2 == 0) {
+        prev0 = a;
+        prev1 = bb;
+      } else {
+        pk[i / 2] = pack4_e4m3(prev0, prev1, a, bb);
+      }
+    } else {
+      pk[i] = pack2<BF16>(a, bb);
+    }
   }
   xp_max = xm;
   return sum0 + sum1;
@@ -1015,7 +1027,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tc_fence_after();
           bool raise = false;
           float alpha = 1.f, m_new = m;
-          if constexpr (kStaleMaxFirst<D>()) {
+          if constexpr (kStaleMaxFirst<D, FP8>()) {
             // S of this tile, keys past the row's last visible key set to -inf
             float s[128];
             auto load_s = [&]() {
@@ -1037,22 +1049,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             load_s();
 
             // P = 2^(s * scale * log2 e - m), packed two keys per 32-bit word
-            // (even key in the low half).  After the first tile the running
-            // max m is tried as it stands: the sum of the tile's P bounds every
-            // P, so if it stays below 2^15 (and every exponent given to the
-            // polynomial lies in its valid range, see exp_row) no P overflows
-            // a 16-bit float and the result is exact with the stale max, and
-            // the row max is never computed.  Otherwise (or on the first
+            // (even key in the low half; e4m3: four per word).  After the
+            // first tile the running max m is tried as it stands: the sum of
+            // the tile's P bounds every P, so if it stays below 2^15 (e4m3:
+            // 448, its largest finite value) and every exponent given to the
+            // polynomial lies in its valid range (see exp_row), no P overflows
+            // its format and the result is exact with the stale max, and the
+            // row max is never computed.  Otherwise (or on the first
             // tile) S is read again and the row max decides, as below.  P is
             // written to TMEM only after that decision, so S is still there
             // to be read again.
-            uint32_t pk[64];
+            uint32_t pk[FP8 ? 32 : 64];
             float tsum = 0.f;
             bool settled = false;
             if (j > 0) {
               float xp_max;
-              tsum = exp_row<D, BF16, true>(s, sl2, -m, pk, xp_max);
-              settled = __all_sync(0xffffffffu, tsum < 32768.f && xp_max < POLY_X_LIMIT);
+              tsum = exp_row<D, BF16, true, FP8>(s, sl2, -m, pk, xp_max);
+              // every P below the largest finite value of its format
+              settled = __all_sync(0xffffffffu,
+                                   tsum < (FP8 ? 448.f : 32768.f) && xp_max < POLY_X_LIMIT);
               if (!settled) load_s();
             }
             if (!settled) {
@@ -1079,10 +1094,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
               const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
               alpha = raise ? ex2_approx(m - m_use) : 1.f;
               float xp_unused;
-              tsum = exp_row<D, BF16, false>(s, sl2, -m_use, pk, xp_unused);
+              tsum = exp_row<D, BF16, false, FP8>(s, sl2, -m_use, pk, xp_unused);
             }
             tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(pk));
-            tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
+            if constexpr (!FP8) tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(pk + 32));
             l = l * alpha + tsum;
             m = m_new;
           } else {

@@ -4,10 +4,11 @@ Reads the coefficients from the CUDA header, replays the kernel's float32
 steps (clamp at -126, round-to-integer by adding 1.5 * 2^23, degree-3
 Horner on the remainder, add the integer to the exponent field) and checks
 the relative error over the range the softmax can produce (x <= 8 with the
-lazy rescale threshold, x >= -126 before the clamp), and, for the d = 64
-stale-max path where x has no upper bound, that the row acceptance rule
-(P sum below 2^15 and every polynomial exponent below the limit read from
-the kernel) never accepts a row holding a wrong or overflowing P.
+lazy rescale threshold, x >= -126 before the clamp), and, for the
+stale-max path (d = 64, and e4m3 operands) where x has no upper bound, that
+the row acceptance rule (P sum below 2^15, or 448 for e4m3, and every
+polynomial exponent below the limit read from the kernel) never accepts a
+row holding a wrong or overflowing P.
 
 These are consistency checks of a restated formula, not kernel evidence:
 the GPU parity tests with planted dominant keys exercise the kernel itself.
@@ -30,8 +31,17 @@ def poly_x_limit():
 
 
 def poly_pairs_d64():
+    """Polynomial pairs per 16 at d = 64 and with e4m3 operands (one constant for both)."""
     text = open(KERNEL, encoding="utf-8").read()
-    return int(re.search(r"exp_poly_pairs\(\) \{ return D == 64 \? ([0-9]+) : 0; \}", text).group(1))
+    return int(re.search(r"exp_poly_pairs\(\) \{ return \(D == 64 \|\| FP8\) \? ([0-9]+) : 0; \}",
+                         text).group(1))
+
+
+def stale_sum_limits():
+    """The two P-sum limits of the stale acceptance: (16-bit, e4m3)."""
+    text = open(KERNEL, encoding="utf-8").read()
+    m = re.search(r"tsum < \(FP8 \? ([0-9.]+)f : ([0-9.]+)f\)", text)
+    return float(m.group(2)), float(m.group(1))
 
 
 def coefficients():
@@ -108,8 +118,8 @@ def _mufu_exp2(x):
     return np.where(x < -126.0, 0.0, y)
 
 
-def _stale_row(x, use_limit=True):
-    """Replay of the stale-max acceptance of one 128-key row (exp_row<64, *, true>)."""
+def _stale_row(x, use_limit=True, fp8=False):
+    """Replay of the stale-max acceptance of one 128-key row (exp_row<D, *, true, FP8>)."""
     pairs = poly_pairs_d64()
     keys = np.arange(128)
     poly = (keys // 2) % 16 < pairs
@@ -117,7 +127,8 @@ def _stale_row(x, use_limit=True):
         p = np.where(poly, kernel_exp2(x).astype(np.float64), _mufu_exp2(x))
     tsum = float(np.sum(p))
     xp_max = float(np.max(x[poly]))
-    accepted = tsum < 32768.0 and (xp_max < poly_x_limit() if use_limit else True)
+    limit = stale_sum_limits()[1 if fp8 else 0]
+    accepted = tsum < limit and (xp_max < poly_x_limit() if use_limit else True)
     return accepted, p
 
 
@@ -145,6 +156,31 @@ def test_stale_acceptance_never_admits_a_wrong_p():
             assert rel.max() < 1.0e-4, (key, gap, rel.max())
         else:
             assert gap >= 15.0, (key, gap)  # rejected rows go to the row-max path
+    assert n > 0
+
+
+def test_stale_limits_are_the_formats_largest_values():
+    """2^15 stays below fp16's largest finite 65504; 448 is e4m3's largest finite value."""
+    assert stale_sum_limits() == (32768.0, 448.0)
+
+
+def test_stale_acceptance_e4m3_keeps_every_p_in_range():
+    """e4m3: an accepted row has every P finite and below 448 (no saturation), within the
+    polynomial's error; a rejected row holds a key whose P alone is at least 448 / 128."""
+    rng = np.random.default_rng(11)
+    n = 0
+    for key, gap, x in _rows_with_one_big_key(rng):
+        for g in (gap, gap - 13.0, 8.0, 8.7, 8.9):
+            x2 = x.copy()
+            x2[key] = np.float32(g)
+            accepted, p = _stale_row(x2, fp8=True)
+            if accepted:
+                n += 1
+                ref = np.exp2(x2.astype(np.float64))
+                assert np.all(np.isfinite(p)) and p.max() < 448.0, (key, g)
+                assert np.abs(p / ref - 1.0).max() < 1.0e-4, (key, g)
+            else:
+                assert g > np.log2(448.0 / 128.0), (key, g)
     assert n > 0
 
 
