@@ -95,14 +95,15 @@ struct BwdSmem {
   static constexpr int DQ_READY = DS_READY + 1;   // dK and dQ of the tile done
   static constexpr int DQ_FREE = DQ_READY + 1;    // 128 readout threads arrive
   static constexpr int DONE = DQ_FREE + 1;        // every MMA done
-  static constexpr int SYNC = DONE + 1;           // rendezvous of the 256 softmax threads
-  static constexpr int RO_SYNC = SYNC + 1;        // rendezvous of the 128 readout threads
+  static constexpr int RO_SYNC = DONE + 1;        // rendezvous of the 128 readout threads
   static constexpr int NUM_BARS = RO_SYNC + 1;
   static constexpr int MISC_OFF = BAR_OFF + NUM_BARS * 8;  // TMEM address, abort flag
   static constexpr int BYTES = MISC_OFF + 16 + 1024;      // + slack to align the base to 1 KB
   static_assert(BYTES <= 232448, "shared memory budget");
   // TMEM columns (512 allocated)
-  static constexpr uint32_t S_COL = 0;     // S^T fp32 [key][query]; P^T 16-bit pairs in [0, 64)
+  // S^T fp32 [key][query]; P^T as 16-bit pairs, queries 64 w .. 64 w + 63 in
+  // columns 64 w .. 64 w + 31 (each warpgroup over the S^T columns it read)
+  static constexpr uint32_t S_COL = 0;
   static constexpr uint32_t DP_COL = 128;  // dP^T fp32; then dQ_ij [query][D] in [128, 128 + D)
   static constexpr uint32_t DK_COL = 256;  // dK [key][D]
   static constexpr uint32_t DV_COL = 256 + D;  // dV [key][D]
@@ -256,7 +257,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     mbar_init(bar(L::DQ_READY), 1);
     mbar_init(bar(L::DQ_FREE), 128);
     mbar_init(bar(L::DONE), 1);
-    mbar_init(bar(L::SYNC), 256);
     mbar_init(bar(L::RO_SYNC), 128);
     *abort_flag = 0;
     fence_mbarrier_init();
@@ -379,15 +379,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         mma_commit(bar(L::DP_READY));
       }
       __syncwarp();
-      // dV += P^T dO_i (P^T from TMEM, 16 queries = 8 columns per k-step)
+      // dV += P^T dO_i (P^T from TMEM, 16 queries = 8 columns per k-step;
+      // queries 64 w .. 64 w + 63 at columns 64 w .. 64 w + 31)
       ok = __all_sync(0xffffffffu, wait_phase(bar(L::P_READY), n & 1, abort_flag, SITE_MMA_P_FULL));
       if (!ok) break;
       tc_fence_after();
       if (leader) {
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_ts(t_dv, t_s + kk * 8, ring_mn + do16 + kk * (2048 >> 4), IDESC_KB,
-                 (n > 0 || kk > 0) ? 1u : 0u);
+          mma_ts(t_dv, t_s + (kk >> 2) * 64 + (kk & 3) * 8, ring_mn + do16 + kk * (2048 >> 4),
+                 IDESC_KB, (n > 0 || kk > 0) ? 1u : 0u);
       }
       __syncwarp();
       // S^T(n + 1): queued behind dV(n), which reads the P^T it overwrites
@@ -536,6 +537,23 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         ds_lo = dsum_bh[qw + lane];
         ds_hi = dsum_bh[qw + 32 + lane];
       }
+      // d = 64: the stage's lse2 / D landed with Q_i; these threads observe
+      // that stage's completed phase themselves before reading them (the
+      // stage is refilled only after this tile's dS is handed over, so the
+      // phase is unambiguous; S^T(n) is computed from the same stage).  The
+      // first lse2 values are loaded before the S wait and each later one
+      // four float4 ahead of its use, so no exponential waits on a load.
+      const float* stage_stats = stats_smem + (n % L::STAGES) * 256;
+      const float4* l4 = reinterpret_cast<const float4*>(stage_stats + 64 * w);
+      float4 lq[4];
+      if constexpr (L::STATS_IN_SMEM) {
+        ok = __all_sync(0xffffffffu, wait_phase(bar(L::RING_FULL + n % L::STAGES),
+                                                (n / L::STAGES) & 1, abort_flag,
+                                                SITE_SOFTMAX_S_FULL));
+        if (!ok) break;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) lq[i] = l4[i];
+      }
       ok = __all_sync(0xffffffffu, wait_phase(bar(L::S_READY), n & 1, abort_flag,
                                               SITE_SOFTMAX_S_FULL));
       if (!ok) break;
@@ -544,33 +562,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tmem_ld32(t_s + 64 * w, *reinterpret_cast<uint32_t(*)[32]>(sr));
       tmem_ld32(t_s + 64 * w + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
       tmem_wait_ld_regs(sr);
-      // P^T is written over S^T columns [0, 64), which hold the other
-      // warpgroup's S until it has read them: both finish reading first
-      // (a bounded mbarrier rendezvous, so an aborted partner cannot hang it)
-      mbar_arrive(bar(L::SYNC));
-      ok = __all_sync(0xffffffffu, wait_phase(bar(L::SYNC), n & 1, abort_flag, SITE_SOFTMAX_SYNC));
-      if (!ok) break;
       // P = 2^(s * scale * log2 e - lse2); 0 for keys past Nk, queries past
       // Nq (lse2 = +inf there) and, causal, queries before the key
       uint32_t pk[32];
-      // the stage's lse2 / D landed with Q_i; these threads observe that
-      // stage's completed phase themselves before reading them (the stage is
-      // refilled only after this tile's dS is handed over, so the phase is
-      // unambiguous and already complete: S^T(n) was computed from it)
-      if constexpr (L::STATS_IN_SMEM) {
-        ok = __all_sync(0xffffffffu, wait_phase(bar(L::RING_FULL + n % L::STAGES),
-                                                (n / L::STAGES) & 1, abort_flag,
-                                                SITE_SOFTMAX_S_FULL));
-        if (!ok) break;
-      }
-      const float* stage_stats = stats_smem + (n % L::STAGES) * 256;
-      const float4* l4 = reinterpret_cast<const float4*>(stage_stats + 64 * w);
       const bool diag = p.causal && qw < key;  // some of these queries precede the key
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
         float lsv[4];
         if constexpr (L::STATS_IN_SMEM) {
-          const float4 lv = l4[c4];
+          const float4 lv = lq[c4 % 4];
+          if (c4 + 4 < 16) lq[c4 % 4] = l4[c4 + 4];
           lsv[0] = lv.x;
           lsv[1] = lv.y;
           lsv[2] = lv.z;
@@ -591,12 +592,20 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         pk[2 * c4] = pack2<BF16>(pv[0], pv[1]);
         pk[2 * c4 + 1] = pack2<BF16>(pv[2], pv[3]);
       }
-      tmem_st16(t_s + 32 * w, *reinterpret_cast<uint32_t(*)[16]>(pk));
-      tmem_st16(t_s + 32 * w + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
+      // over this warpgroup's own S^T columns, which only it has read
+      tmem_st16(t_s + 64 * w, *reinterpret_cast<uint32_t(*)[16]>(pk));
+      tmem_st16(t_s + 64 * w + 16, *reinterpret_cast<uint32_t(*)[16]>(pk + 16));
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(L::P_READY));
-      // dS = P (dP - D), from the rounded P the dV product used
+      // dS = P (dP - D), from the rounded P the dV product used; the D values
+      // are loaded ahead of their use like lse2
+      const float4* d4 = reinterpret_cast<const float4*>(stage_stats + 128 + 64 * w);
+      float4 dq4[4];
+      if constexpr (L::STATS_IN_SMEM) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) dq4[i] = d4[i];
+      }
       ok = __all_sync(0xffffffffu, wait_phase(bar(L::DP_READY), n & 1, abort_flag,
                                               SITE_SOFTMAX_S_FULL));
       if (!ok) break;
@@ -606,7 +615,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         if (!ok) break;
       }
       tc_fence_after();
-      const float4* d4 = reinterpret_cast<const float4*>(stage_stats + 128 + 64 * w);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         uint32_t dp[32];
@@ -617,7 +625,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         for (int c4 = 0; c4 < 8; ++c4) {
           float dsv[4];
           if constexpr (L::STATS_IN_SMEM) {
-            const float4 dv = d4[8 * half + c4];
+            const int di = 8 * half + c4;
+            const float4 dv = dq4[di % 4];
+            if (di + 4 < 16) dq4[di % 4] = d4[di + 4];
             dsv[0] = dv.x;
             dsv[1] = dv.y;
             dsv[2] = dv.z;
