@@ -18,11 +18,15 @@
 // into the producing and consuming GEMMs, which is where the extra HBM
 // round trips of the unfused block are.
 //
-// One CTA per 128 x 128 output tile; K in 64-wide steps through a 4-stage
+// One CTA per 128 x 128 output tile; K in 64-wide steps through a 2-stage
 // TMA ring (128-byte swizzle, both operands K-major, the layout and
 // descriptors of the attention kernel's S = Q K^T); warp 4 loads, warp 5
 // issues tcgen05.mma (fp32 accumulator in TMEM), warps 0-3 read the
-// accumulator back (one row per thread), add the bias and store.
+// accumulator back (one row per thread), add the bias and store.  With K as
+// short as the block's channel count (256 .. 1024) a tile is mostly load
+// latency and epilogue, so the ring is kept small enough (65 KB) for three
+// CTAs per SM: one CTA's epilogue and start-up overlap the others' loads and
+// MMAs (4 stages and one CTA per SM took 35-50 % longer).
 #pragma once
 
 #include <cstdint>
@@ -34,7 +38,8 @@
 namespace attn_sm100 {
 
 constexpr int PROJ_THREADS = 192;
-constexpr int PROJ_STAGES = 4;
+constexpr int PROJ_STAGES = 2;
+constexpr int PROJ_CTAS_PER_SM = 3;  // shared memory 3 x 65 KB, TMEM 3 x 128 columns
 constexpr int PROJ_LOAD_WARP = 4;
 constexpr int PROJ_MMA_WARP = 5;
 
@@ -65,7 +70,7 @@ struct ProjSmem {
 };
 
 template <bool BF16, int MODE>
-__global__ void __launch_bounds__(PROJ_THREADS, 1)
+__global__ void __launch_bounds__(PROJ_THREADS, PROJ_CTAS_PER_SM)
     proj_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                      const ProjParams p) {
   using L = ProjSmem;
