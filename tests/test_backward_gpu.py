@@ -187,3 +187,70 @@ def test_backward_repeatable_dk_dv():
     _, dk2, dv2 = A.backward(q, k, v, o, lse, do, causal=True)
     torch.cuda.synchronize()
     assert torch.equal(dk1, dk2) and torch.equal(dv1, dv2)
+
+
+def _sampled_head(q, k, v, do, o, lse, scale, causal, u, keys, queries):
+    """dK, dV of the sampled keys and dQ of the sampled queries of one (batch, head), from the
+    oracle's steps on the kernel's saved o and lse, with the per-element bounds of _bounds.
+
+    A key's dK and dV need its column of P over every query and a query's dQ its row over every
+    key, so each sample is a slice of the definition computed whole."""
+    nq = q.shape[0]
+    qi = np.arange(nq)
+    D = row_dot(do, o)
+    # columns: every query against the sampled keys
+    s_c = scores(q, k[keys], scale)
+    if causal:
+        s_c = np.where(keys[None, :] > qi[:, None], -np.inf, s_c)
+    p_c = recompute_probs(s_c, lse)
+    dp_c = grad_p(do, v[keys])
+    ds_c = grad_scores(p_c, dp_c, D)
+    dv = p_c.T @ do
+    dk = scale * (ds_c.T @ q)
+    e32_c = 2.0 ** -22 * np.abs(p_c) * (np.abs(do) @ np.abs(v[keys]).T + row_dot(np.abs(do), np.abs(o))[:, None])
+    b_dv = 2 * u * (np.abs(p_c).T @ np.abs(do))
+    b_dk = scale * (2 * u * (np.abs(ds_c).T @ np.abs(q)) + e32_c.T @ np.abs(q))
+    # rows: the sampled queries against every key
+    s_r = scores(q[queries], k, scale)
+    if causal:
+        s_r = apply_causal_mask(s_r, queries)
+    p_r = recompute_probs(s_r, lse[queries])
+    ds_r = grad_scores(p_r, grad_p(do[queries], v), D[queries])
+    dq = scale * (ds_r @ k)
+    e32_r = 2.0 ** -22 * np.abs(p_r) * (np.abs(do[queries]) @ np.abs(v).T + row_dot(np.abs(do[queries]), np.abs(o[queries]))[:, None])
+    b_dq = scale * (2 * u * (np.abs(ds_r) @ np.abs(k)) + e32_r @ np.abs(k))
+    return (dq, b_dq), (dk, b_dk), (dv, b_dv)
+
+
+@pytest.mark.parametrize("idx", [2, 3, 4])
+def test_backward_workloads_full_size_sampled(idx):
+    """The 80x80, causal 2048 and 32k workloads at full size, in the launch bench.py times:
+    dK and dV of 48 keys (the first and last 16 and 16 seeded ones) and dQ of 48 queries chosen
+    the same way, in four (batch, head) slices, against the oracle's steps with the derived
+    per-element bounds (the floor taken over the sampled elements)."""
+    w = WORKLOADS[idx]
+    q, k, v = make_workload_qkv(w)
+    do = make_grad_out(w.B, w.H, w.Nq, w.d, w.dtype, w.seed)
+    o, lse, dq, dk, dv = _gpu_forward_backward(q, k, v, do, w.causal, w.scale)
+    u = UNIT[w.dtype]
+    rng = np.random.default_rng(idx)
+    bh = w.B * w.H
+    heads = sorted({0, bh - 1} | set(int(x) for x in rng.integers(0, bh, 2)))
+    worst = {"dq": 0.0, "dk": 0.0, "dv": 0.0}
+
+    def pick(n):
+        return np.unique(np.concatenate([np.arange(16), np.arange(n - 16, n), rng.integers(16, n - 16, 16)]))
+    for flat in heads:
+        b, h = divmod(flat, w.H)
+        keys, queries = pick(w.Nk), pick(w.Nq)
+        res = _sampled_head(_f64(q[b, h]), _f64(k[b, h]), _f64(v[b, h]), _f64(do[b, h]),
+                            _f64(o[b, h]), _f64(lse[b, h]), w.scale, w.causal, u, keys, queries)
+        got = {"dq": _f64(dq[b, h])[queries], "dk": _f64(dk[b, h])[keys], "dv": _f64(dv[b, h])[keys]}
+        for name, (r, bnd) in zip(("dq", "dk", "dv"), res):
+            g = got[name]
+            assert np.all(np.isfinite(g)), f"{name} not finite at ({b},{h})"
+            tol = 2 * (bnd + u * np.abs(r)) + 2.0 ** -20 * (np.max(np.abs(r)) + 1e-30)
+            ratio = float(np.max(np.abs(g - r) / tol))
+            worst[name] = max(worst[name], ratio)
+            assert ratio <= 1.0, f"{name} ({b},{h}): err/tol {ratio:.3f}"
+    print(f"\nBWD SAMPLED {w.name}: max err/tol " + ", ".join(f"{n} {r:.3f}" for n, r in worst.items()))

@@ -464,3 +464,22 @@ def test_host_entry_pipelined_matches_device_entry(B, H, N, d, dtype, causal, wi
     if with_lse:
         assert torch.equal(lh, lse.cpu())
     assert A.attn_get_device_status()[0] == 0
+
+
+@pytest.mark.parametrize("dtype,causal", [("bf16", True), ("fp16", False)])
+def test_128k_context_sampled(dtype, causal):
+    """The longest context the pages speak of (128K tokens, FA3 on a 70B model): one
+    (batch, head) pair per head of B = 1, H = 2, N = 131072, d = 128, Q and K x 0.5 like the
+    long-context workload.  The first, 32 seeded and the last 32 query rows of each head against
+    all 131072 keys, within the forward's bars."""
+    B, H, N, d = 1, 2, 131072, 128
+    q, k, v = make_qkv(B, H, N, N, d, dtype, seed=131, qk_scale=0.5)
+    scale = 1.0 / math.sqrt(d)
+    o, lse = _run(q, k, v, causal, scale)
+    rng = np.random.default_rng(131)
+    rows = np.unique(np.concatenate([np.arange(32), rng.integers(32, N - 32, 32), np.arange(N - 32, N)]))
+    for h in range(H):
+        o_ref, l_ref = oracle.attention_head_rows(q[0, h, rows], k[0, h], v[0, h], scale, causal, rows)
+        assert _err(o[0, h, rows].double().numpy(), o_ref) <= TOL[dtype]
+        assert _err(lse[0, h, rows].double().numpy(), l_ref) <= LSE_TOL
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
