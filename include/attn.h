@@ -74,8 +74,9 @@ typedef struct {
                         each pair the lone last query tile of two heads; else 0            */
   int grid;          /* persistent CTAs launched: min(num_units, SM count)                */
   int block;         /* threads per CTA                                                   */
-  int smem_bytes;    /* dynamic shared memory per CTA                                     */
-  int stages;        /* K/V shared-memory ring slots                                      */
+  int smem_bytes;    /* dynamic shared memory per CTA (16-bit operands; attn_fwd_fp8's
+                        e4m3 tiles take 4 + 4 ring slots and about 193 KB)                 */
+  int stages;        /* K/V shared-memory ring slots (16-bit operands)                    */
   long long qk_tile_products; /* 128x128 score tiles computed (incl. masked tail tiles)   */
   int split;         /* 1 if attn_fwd_ws would use split mode for these sizes (see below)  */
   int split_grid;    /* CTAs launched in split mode: min(SM count, split_steps)             */
