@@ -173,9 +173,12 @@ __global__ void __launch_bounds__(PROJ_THREADS, PROJ_CTAS_PER_SM)
       tc_fence_after();
       long long row;  // PROJ_QKV: row of x (b N + n); PROJ_OUT: n within batch b_out
       bool row_ok;
+      long long qkv_b = 0, qkv_n = 0;  // PROJ_QKV: the row's batch and position, split once
       if constexpr (MODE == PROJ_QKV) {
         row = static_cast<long long>(m_tile) * 128 + r;
         row_ok = row < static_cast<long long>(p.B) * p.N;
+        qkv_b = row / p.N;
+        qkv_n = row - qkv_b * p.N;
       } else {
         row = n0_out + r;
         row_ok = row < p.N;
@@ -203,7 +206,7 @@ __global__ void __launch_bounds__(PROJ_THREADS, PROJ_CTAS_PER_SM)
           const int C = p.H * p.d;
           const int which = col0 / C, rem = col0 - which * C;
           const int h = rem / p.d, dd = rem - h * p.d;
-          const long long b = row / p.N, n = row - b * p.N;
+          const long long b = qkv_b, n = qkv_n;
           void* base = which == 0 ? p.out0 : (which == 1 ? p.out1 : p.out2);
           dst = static_cast<uint16_t*>(base) + ((b * p.H + h) * p.N + n) * p.d + dd;
         } else {
