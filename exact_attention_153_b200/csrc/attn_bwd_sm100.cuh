@@ -20,8 +20,8 @@
 //     P^T (written back over S^T as 16-bit pairs) and dS^T (written to a
 //     128-byte-swizzled shared-memory tile), and the tensor core accumulates
 //     dV += P^T dO_i and dK += dS^T Q_i in TMEM and computes dQ_ij = dS K_j,
-//     which a readout warpgroup adds into the fp32 dQ accumulator with
-//     vector atomics;
+//     which a readout warpgroup stages in shared memory and adds into the
+//     fp32 dQ accumulator with TMA bulk reductions;
 //   * bwd_dq_kernel: dQ = scale * accumulator, rounded to the input dtype.
 //
 // Every operand layout is one the forward already uses: K-major tiles as the
