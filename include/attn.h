@@ -87,6 +87,14 @@ typedef struct {
 } attn_plan_t;
 
 /*
+ * CUDA graphs.  attn_fwd, attn_fwd_ws, attn_fwd_fp8, attn_bwd, attn_qkv_proj, attn_out_proj and
+ * attn_block_fwd allocate nothing and never synchronise, so after one ordinary call with the
+ * same dtype and head size (which sets the kernel's shared-memory attribute) they can be
+ * captured into a CUDA graph on the caller's stream and replayed; split mode resets its piece
+ * counters at the end of every call, so a captured workspace stays valid across replays.
+ */
+
+/*
  * attn_fwd -- the attention forward on device memory.
  *
  *   q, k, v  device pointers, 16-byte aligned, layouts above, read only.
