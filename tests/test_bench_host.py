@@ -57,3 +57,15 @@ def test_both_arms_print_the_same_config(capsys, monkeypatch):
 def test_percentiles():
     st = bench.percentiles([float(x) for x in range(1, 101)])
     assert st["median"] == 50.5 and abs(st["p10"] - 10.9) < 1e-9 and abs(st["p90"] - 90.1) < 1e-9
+
+
+def test_fp8_configs_fit_the_entry_point():
+    """The FP8 leg's shapes meet attn_fwd_fp8's rules (d = 128 is implied; Nk a multiple of 16),
+    the long-context one matches the bf16 long-context workload, and --part fp8 finds a config
+    for every workload name."""
+    for name, B, H, N, causal, qk in bench.FP8_CONFIGS:
+        assert N % 16 == 0 and B >= 1 and H >= 1
+    w = workload("long_context_32k")
+    _, B, H, N, causal, qk = bench.fp8_config("long_context_32k")
+    assert (B, H, N, causal, qk) == (w.B, w.H, w.Nq, w.causal, w.qk_scale) and w.d == 128
+    assert bench.fp8_config("yolo_highres_80x80_b16_d128")[2:4] == (2, 6400)
